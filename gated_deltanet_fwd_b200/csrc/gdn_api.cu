@@ -1,0 +1,187 @@
+// gdn_api.cu -- the exported C ABI (include/gdn.h): host-side argument checks, then one launch.
+//
+// Every check happens before anything is enqueued, so a rejected call leaves the stream
+// untouched.  Device-side faults are reported through the workspace status word (chunk prefill)
+// and never trap.
+#include <stdio.h>
+
+#include "gdn_internal.cuh"
+
+using namespace gdn;
+
+namespace {
+
+inline cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
+
+inline bool bad_dtype(gdn_dtype d) { return d != GDN_BF16 && d != GDN_F32; }
+
+inline gdn_status from_cuda(cudaError_t e) { return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA; }
+
+// Pointers that must be present and 16-byte aligned.
+inline bool ptr_ok(const void* p) { return p != nullptr && aligned16(p); }
+
+constexpr size_t kStatusBytes = 256;  // status word + padding to keep the workspace aligned
+
+}  // namespace
+
+extern "C" {
+
+const char* gdn_status_string(gdn_status s) {
+  switch (s) {
+    case GDN_OK: return "GDN_OK";
+    case GDN_ERR_INVALID_ARG: return "GDN_ERR_INVALID_ARG: invalid argument";
+    case GDN_ERR_UNSUPPORTED: return "GDN_ERR_UNSUPPORTED: shape or dtype not implemented";
+    case GDN_ERR_CUDA: return "GDN_ERR_CUDA: CUDA runtime or launch failure";
+    case GDN_ERR_TIMEOUT: return "GDN_ERR_TIMEOUT: a device-side wait ran out";
+    case GDN_ERR_DEVICE_ARG: return "GDN_ERR_DEVICE_ARG: a kernel found a bad device argument";
+  }
+  return "unknown gdn_status";
+}
+
+gdn_status gdn_gates(const void* a, const void* b, gdn_dtype ab_dtype, const float* A_log,
+                     const float* dt_bias, int64_t n_tok, int Hv, float* g, float* beta,
+                     void* stream) {
+  if (bad_dtype(ab_dtype) || n_tok < 0 || Hv < 1) return GDN_ERR_INVALID_ARG;
+  if (n_tok == 0) return GDN_OK;
+  if (!a || !b || !A_log || !dt_bias || !g || !beta) return GDN_ERR_INVALID_ARG;
+  return from_cuda(launch_gates(a, b, ab_dtype, A_log, dt_bias, n_tok, Hv, g, beta,
+                                as_stream(stream)));
+}
+
+gdn_status gdn_causal_conv1d_silu(const void* x, gdn_dtype dtype, const float* w,
+                                  const float* bias, int B, int64_t T, int C, int K,
+                                  const int32_t* cu_seqlens, int N, int n_l2norm_ch,
+                                  int l2norm_group, float l2_eps, const float* conv_state_in,
+                                  float* conv_state_out, void* y, void* stream) {
+  if (bad_dtype(dtype) || B < 0 || T < 0 || C < 1 || K < 1 || N < 0) return GDN_ERR_INVALID_ARG;
+  if (cu_seqlens ? (B != 1 && !(B == 0 && T == 0)) : (N != B)) return GDN_ERR_INVALID_ARG;
+  if (n_l2norm_ch < 0 || n_l2norm_ch > C || l2norm_group < 0) return GDN_ERR_INVALID_ARG;
+  if (!(l2_eps >= 0.0f)) return GDN_ERR_INVALID_ARG;
+  if (K > 8 || C % 8 != 0) return GDN_ERR_UNSUPPORTED;
+  if (l2norm_group != 0 && l2norm_group != 32 && l2norm_group != 64 && l2norm_group != 128 &&
+      l2norm_group != 256)
+    return GDN_ERR_UNSUPPORTED;
+  if (l2norm_group == 0 ? n_l2norm_ch != 0 : n_l2norm_ch % l2norm_group != 0)
+    return GDN_ERR_INVALID_ARG;
+  const int64_t n_tok = (int64_t)B * T;
+  if (cu_seqlens && n_tok > 0 && N < 1) return GDN_ERR_INVALID_ARG;
+  if (n_tok == 0 && (N == 0 || !conv_state_out)) return GDN_OK;
+  if (!w) return GDN_ERR_INVALID_ARG;
+  if (n_tok > 0 && (!ptr_ok(x) || !ptr_ok(y))) return GDN_ERR_INVALID_ARG;
+  if (n_tok > 0) {
+    const size_t eb = dtype == GDN_BF16 ? 2 : 4;
+    const char* xb = (const char*)x;
+    const char* yb = (const char*)y;
+    const size_t bytes = (size_t)n_tok * C * eb;
+    if (xb < yb + bytes && yb < xb + bytes) return GDN_ERR_INVALID_ARG;  // x, y overlap
+  }
+  if (conv_state_in && conv_state_out && K > 1) {
+    const size_t bytes = (size_t)N * C * (K - 1) * sizeof(float);
+    const char* i0 = (const char*)conv_state_in;
+    const char* o0 = (const char*)conv_state_out;
+    if (i0 < o0 + bytes && o0 < i0 + bytes) return GDN_ERR_INVALID_ARG;
+  }
+  cudaStream_t s = as_stream(stream);
+  if (n_tok == 0) {
+    // every sequence is empty: the state passes through unchanged
+    if (K == 1) return GDN_OK;
+    const size_t bytes = (size_t)N * C * (K - 1) * sizeof(float);
+    if (conv_state_in)
+      return from_cuda(cudaMemcpyAsync(conv_state_out, conv_state_in, bytes,
+                                       cudaMemcpyDeviceToDevice, s));
+    return from_cuda(cudaMemsetAsync(conv_state_out, 0, bytes, s));
+  }
+  return from_cuda(launch_conv(x, dtype, w, bias, B, T, C, K, cu_seqlens, N, n_l2norm_ch,
+                               l2norm_group, l2_eps, conv_state_in,
+                               K > 1 ? conv_state_out : nullptr, y, s));
+}
+
+size_t gdn_chunk_fwd_workspace_size(int N, int B, int64_t T, int Hk, int Hv, int dk, int dv,
+                                    int chunk) {
+  (void)N; (void)B; (void)T; (void)Hk; (void)Hv; (void)dk; (void)dv; (void)chunk;
+  return kStatusBytes;
+}
+
+gdn_status gdn_workspace_status(const void* workspace, void* stream, int* device_status) {
+  if (!workspace || !device_status) return GDN_ERR_INVALID_ARG;
+  int v = -1;
+  cudaStream_t s = as_stream(stream);
+  if (cudaMemcpyAsync(&v, workspace, sizeof(int), cudaMemcpyDeviceToHost, s) != cudaSuccess)
+    return GDN_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return GDN_ERR_CUDA;
+  *device_status = v;
+  return GDN_OK;
+}
+
+gdn_status gdn_chunk_fwd(const void* q, const void* k, const void* v, const float* g,
+                         const float* beta, gdn_dtype dtype, float scale,
+                         const float* initial_state, const int32_t* cu_seqlens, int N, int B,
+                         int64_t T, int Hk, int Hv, int dk, int dv, int chunk, void* out,
+                         float* final_state, void* workspace, size_t workspace_bytes,
+                         void* stream) {
+  if (bad_dtype(dtype) || N < 0 || B < 0 || T < 0 || Hk < 1 || Hv < 1 || dk < 1 || dv < 1)
+    return GDN_ERR_INVALID_ARG;
+  if (Hv % Hk != 0) return GDN_ERR_INVALID_ARG;
+  if (cu_seqlens ? (B != 1) : (N != B)) return GDN_ERR_INVALID_ARG;
+  if (!(scale == scale)) return GDN_ERR_INVALID_ARG;  // NaN
+  if (dk % 16 != 0 || dv % 16 != 0 || dk > 128 || dv > 128) return GDN_ERR_UNSUPPORTED;
+  if (chunk != 16 && chunk != 32 && chunk != 64) return GDN_ERR_UNSUPPORTED;
+  if (!workspace || workspace_bytes < gdn_chunk_fwd_workspace_size(N, B, T, Hk, Hv, dk, dv, chunk))
+    return GDN_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return GDN_ERR_INVALID_ARG;
+  if (N == 0) return GDN_OK;
+  const int64_t n_tok = (int64_t)B * T;
+  if (n_tok > 0 && (!ptr_ok(q) || !ptr_ok(k) || !ptr_ok(v) || !ptr_ok(g) || !ptr_ok(beta) ||
+                    !ptr_ok(out)))
+    return GDN_ERR_INVALID_ARG;
+  if ((initial_state && !aligned16(initial_state)) || (final_state && !aligned16(final_state)))
+    return GDN_ERR_INVALID_ARG;
+  if (cu_seqlens && ((uintptr_t)cu_seqlens & 3u)) return GDN_ERR_INVALID_ARG;
+  if (initial_state && final_state) {
+    const size_t bytes = (size_t)N * Hv * dv * dk * sizeof(float);
+    const char* i0 = (const char*)initial_state;
+    const char* o0 = (const char*)final_state;
+    if (i0 < o0 + bytes && o0 < i0 + bytes) return GDN_ERR_INVALID_ARG;
+  }
+  cudaStream_t s = as_stream(stream);
+  int* status = reinterpret_cast<int*>(workspace);
+  if (cudaMemsetAsync(status, 0, sizeof(int), s) != cudaSuccess) return GDN_ERR_CUDA;
+  cudaError_t e;
+  e = launch_chunk_simt(q, k, v, g, beta, dtype, scale, initial_state, cu_seqlens, N, B, T, Hk,
+                          Hv, dk, dv, chunk, out, final_state, status, s);
+  return from_cuda(e);
+}
+
+gdn_status gdn_recurrent_step(const void* q, const void* k, const void* v, const float* g,
+                              const float* beta, gdn_dtype dtype, float scale, float* state,
+                              int N, int Hk, int Hv, int dk, int dv, void* out, void* stream) {
+  if (bad_dtype(dtype) || N < 0 || Hk < 1 || Hv < 1 || dk < 1 || dv < 1)
+    return GDN_ERR_INVALID_ARG;
+  if (Hv % Hk != 0) return GDN_ERR_INVALID_ARG;
+  if (!(scale == scale)) return GDN_ERR_INVALID_ARG;
+  if (dk != 128 || dv % 8 != 0 || dv > 256) return GDN_ERR_UNSUPPORTED;
+  if (N == 0) return GDN_OK;
+  if (!ptr_ok(q) || !ptr_ok(k) || !ptr_ok(v) || !ptr_ok(g) || !ptr_ok(beta) || !ptr_ok(state) ||
+      !ptr_ok(out))
+    return GDN_ERR_INVALID_ARG;
+  return from_cuda(launch_recurrent(q, k, v, g, beta, dtype, scale, state, N, Hk, Hv, dk, dv, out,
+                                    as_stream(stream)));
+}
+
+gdn_status gdn_gated_rmsnorm(const void* x, const void* z, gdn_dtype dtype, const float* w,
+                             float eps, int64_t n_rows, int dim, void* y, void* stream) {
+  if (bad_dtype(dtype) || n_rows < 0 || dim < 1 || !(eps >= 0.0f)) return GDN_ERR_INVALID_ARG;
+  if (dim != 8 && dim != 16 && dim != 32 && dim != 64 && dim != 128 && dim != 256)
+    return GDN_ERR_UNSUPPORTED;
+  if (n_rows == 0) return GDN_OK;
+  if (!ptr_ok(x) || !ptr_ok(z) || !ptr_ok(y) || !w) return GDN_ERR_INVALID_ARG;
+  {
+    const size_t bytes = (size_t)n_rows * dim * (dtype == GDN_BF16 ? 2 : 4);
+    const char* zb = (const char*)z;
+    const char* yb = (const char*)y;
+    if (zb < yb + bytes && yb < zb + bytes) return GDN_ERR_INVALID_ARG;  // y may alias x only
+  }
+  return from_cuda(launch_rmsnorm(x, z, dtype, w, eps, n_rows, dim, y, as_stream(stream)));
+}
+
+}  // extern "C"

@@ -157,7 +157,7 @@ gdn_status gdn_recurrent_step(const void* q, const void* k, const void* v, const
  * of core_attn_out fuses the z gate in, "like SwiGLU").
  *     y[r,j] = x[r,j] * rsqrt(mean_j x[r,.]^2 + eps) * (1 + w[j]) * silu(z[r,j])
  * x, z, y : [n_rows, dim] dtype (e.g. n_rows = B*T*Hv, dim = dv).   w: [dim] fp32.
- * Supported: dim a multiple of 8, 8 <= dim <= 1024; x, z, y 16-byte aligned.  n_rows = 0 launches
+ * Supported: dim in {8, 16, 32, 64, 128, 256}; x, z, y 16-byte aligned.  n_rows = 0 launches
  * nothing.  y may alias x (in place) but not z.
  */
 gdn_status gdn_gated_rmsnorm(const void* x, const void* z, gdn_dtype dtype, const float* w,

@@ -1,0 +1,137 @@
+"""GPU parity of gdn_chunk_fwd (chunked prefill) against the fp64 oracle.
+
+Small cases are compared element by element on every output; the full-size workloads run in the
+launch configuration the bench times and are compared on sampled (sequence, v-head) units, each of
+which the oracle can compute on its own.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from gated_deltanet_fwd_b200 import gdn, inputs
+from gdn_testutil import (assert_bf16_close, assert_f32_close, oracle_gates_f32, oracle_units,
+                          rel_l2)
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+def _gpu_chunk(x, g, beta, chunk, scale):
+    cu = x["cu_seqlens"]
+    S0 = x["initial_state"]
+    out, S = gdn.gdn_chunk_fwd(x["q"].to(DEV), x["k"].to(DEV), x["v"].to(DEV), g.to(DEV),
+                               beta.to(DEV), scale=scale,
+                               initial_state=None if S0 is None else S0.to(DEV),
+                               cu_seqlens=None if cu is None else cu.to(DEV), chunk=chunk)
+    torch.cuda.synchronize()
+    return out.cpu(), S.cpu()
+
+
+def _full_oracle(x, g, beta, scale):
+    return oracle.gated_delta_rule(x["q"], x["k"], x["v"], g, beta, scale,
+                                   initial_state=x["initial_state"],
+                                   cu_seqlens=x["cu_seqlens"], nthreads=8)
+
+
+def _check(dtype, out, S, o_ref, S_ref, what):
+    if dtype == "bf16":
+        assert_bf16_close(out, o_ref, what + " out")
+        assert_bf16_close(S, S_ref, what + " state")
+    else:
+        assert_f32_close(out, o_ref, what + " out")
+        assert_f32_close(S, S_ref, what + " state")
+
+
+def test_tiny_f32_workload():
+    """The tiny all-fp32 check: B=1, T=64, 2 heads, d=16, chunk 16, zero initial state."""
+    w = inputs.WORKLOADS["tiny_f32"]
+    x = inputs.rule_inputs(**w, seed=1000 + w["index"])
+    g, beta = oracle_gates_f32(x)
+    out, S = _gpu_chunk(x, g, beta, w["chunk"], w["dk"] ** -0.5)
+    o_ref, S_ref = _full_oracle(x, g, beta, w["dk"] ** -0.5)
+    _check("f32", out, S, o_ref, S_ref, "tiny")
+
+
+CASES = [
+    # B, T, Hk, Hv, dk, dv, chunk, dtype, seqlens, s0, a_mean
+    (1, 200, 1, 2, 128, 128, 64, "bf16", None, 0.02, 0.0),   # tensor-core shape, ragged tail
+    (2, 130, 2, 4, 128, 128, 64, "bf16", None, None, -6.0),  # slow decay, batch rows
+    (1, 333, 2, 4, 128, 128, 64, "bf16", [1, 64, 0, 65, 127, 76], 0.02, -6.0),  # varlen
+    (1, 96, 2, 2, 128, 128, 64, "bf16", None, 0.05, -6.0),   # Hk == Hv
+    (1, 150, 1, 2, 128, 128, 32, "bf16", None, 0.02, -6.0),  # CUDA-core path, bf16
+    (1, 150, 1, 2, 128, 128, 16, "f32", None, 0.02, -6.0),   # all fp32
+    (1, 100, 2, 4, 64, 32, 64, "f32", [37, 0, 63], 0.1, -6.0),
+    (1, 81, 1, 1, 16, 48, 16, "f32", None, 0.1, -3.0),
+    (1, 70, 1, 2, 128, 64, 64, "bf16", None, 0.02, -6.0),    # dk != dv
+]
+
+
+@pytest.mark.parametrize("case", CASES)
+def test_chunk_small_cases(case):
+    B, T, Hk, Hv, dk, dv, chunk, dtype, seqlens, s0, a_mean = case
+    x = inputs.rule_inputs(B=B, T=T, Hk=Hk, Hv=Hv, dk=dk, dv=dv, dtype=dtype, seed=T + dk,
+                           seqlens=seqlens, s0_std=s0, a_mean=a_mean)
+    g, beta = oracle_gates_f32(x)
+    out, S = _gpu_chunk(x, g, beta, chunk, dk ** -0.5)
+    o_ref, S_ref = _full_oracle(x, g, beta, dk ** -0.5)
+    _check(dtype, out, S, o_ref, S_ref, str(case))
+
+
+def test_chunk_zero_decay():
+    """g = 0 (no forgetting): nothing damps an error carried between chunks."""
+    x = inputs.rule_inputs(B=1, T=256, Hk=1, Hv=2, dk=128, dv=128, seed=4, s0_std=0.02)
+    g, beta = oracle_gates_f32(x)
+    g = torch.zeros_like(g)
+    out, S = _gpu_chunk(x, g, beta, 64, 128 ** -0.5)
+    o_ref, S_ref = _full_oracle(x, g, beta, 128 ** -0.5)
+    _check("bf16", out, S, o_ref, S_ref, "g=0")
+
+
+def test_chunk_empty_and_no_state():
+    """A zero-length sequence returns its initial state; a NULL initial state means zeros."""
+    x = inputs.rule_inputs(B=1, T=64, Hk=1, Hv=2, dk=128, dv=128, seed=9, seqlens=[0, 64],
+                           s0_std=0.02)
+    g, beta = oracle_gates_f32(x)
+    out, S = _gpu_chunk(x, g, beta, 64, 0.1)
+    assert torch.equal(S[0], x["initial_state"][0])
+    x["initial_state"] = None
+    out, S = _gpu_chunk(x, g, beta, 64, 0.1)
+    o_ref, S_ref = _full_oracle(x, g, beta, 0.1)
+    _check("bf16", out, S, o_ref, S_ref, "no S0")
+
+
+def _sampled(wname, units, a_mean=0.0):
+    w = inputs.WORKLOADS[wname]
+    x = inputs.rule_inputs(**w, seed=1000 + w["index"], a_mean=a_mean)
+    g, beta = oracle_gates_f32(x)
+    scale = w["dk"] ** -0.5
+    out, S = _gpu_chunk(x, g, beta, w["chunk"], scale)
+    ref = oracle_units(x["q"], x["k"], x["v"], g, beta, scale, x["initial_state"],
+                       x["cu_seqlens"], units)
+    cu = x["cu_seqlens"]
+    for (n, h), (o_ref, S_ref) in ref.items():
+        if cu is not None:
+            o = out[0, int(cu[n]):int(cu[n + 1]), h]
+        else:
+            o = out[n, :, h]
+        assert_bf16_close(o, o_ref, f"{wname} unit {(n, h)} out")
+        assert_bf16_close(S[n, h], S_ref, f"{wname} unit {(n, h)} state")
+
+
+def test_prefill_4k_sampled():
+    """B=1, T=4096, 16 q/k heads, 32 v heads, d=128, bf16, chunk 64, zero initial state."""
+    _sampled("prefill_4k", [(0, 0), (0, 1), (0, 17), (0, 31)])
+
+
+def test_prefill_4k_slow_decay_sampled():
+    _sampled("prefill_4k", [(0, 3), (0, 30)], a_mean=-6.0)
+
+
+def test_prefill_varlen_32k_sampled():
+    """32768 tokens as 4 sequences (16384/8192/6144/2048) with per-sequence initial states."""
+    _sampled("prefill_varlen_32k", [(0, 0), (1, 9), (2, 20), (3, 31)])
+
+
+def test_prefill_varlen_32k_slow_decay_sampled():
+    _sampled("prefill_varlen_32k", [(0, 5), (3, 16)], a_mean=-6.0)
