@@ -32,6 +32,8 @@ SIGNATURES = {
                                     _P, _P]),
     "gdn_chunk_fwd": (_I, [_P, _P, _P, _P, _P, _I, _F, _P, _P, _I, _I, _I64, _I, _I, _I, _I, _I,
                            _P, _P, _P, _SZ, _P]),
+    "gdn_chunk_fwd_noalloc": (_I, [_P, _P, _P, _P, _P, _I, _F, _P, _P, _I, _I, _I64, _I, _I, _I,
+                                   _I, _I, _P, _P, _P]),
     "gdn_chunk_fwd_workspace_size": (_SZ, [_I, _I, _I64, _I, _I, _I, _I, _I]),
     "gdn_workspace_status": (_I, [_P, _P, ctypes.POINTER(_I)]),
     "gdn_recurrent_step": (_I, [_P, _P, _P, _P, _P, _I, _F, _P, _I, _I, _I, _I, _I, _P, _P]),

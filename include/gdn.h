@@ -126,6 +126,32 @@ gdn_status gdn_chunk_fwd(const void* q, const void* k, const void* v, const floa
                          float* final_state, void* workspace, size_t workspace_bytes,
                          void* stream);
 
+/*
+ * gdn_chunk_fwd_noalloc -- gdn_chunk_fwd for callers that cannot allocate device memory.  The
+ * pages have no counterpart: this is a library convenience.
+ * Who needs it: code that receives device pointers from another runtime and may not allocate
+ * during a call -- e.g. a plugin inside an inference engine that plans all device memory ahead
+ * (cudaMalloc can synchronise the device and stall the engine's other streams), or a host with a
+ * fixed device-memory budget that owns every buffer.  Such callers cannot supply a workspace.
+ * Same arguments, layouts and results as gdn_chunk_fwd, without workspace / workspace_bytes: the
+ * scratch is a fixed array of GDN_NOALLOC_SCRATCH_BYTES inside the library (a __device__
+ * variable that every GPU which loads the library holds until the process exits).  Sizes whose
+ * gdn_chunk_fwd_workspace_size() exceeds that maximum return GDN_ERR_UNSUPPORTED.  The call
+ * allocates nothing (no cudaMalloc, cudaFree or allocating library routine).
+ * The first call on each device looks up the array's device address (cudaGetSymbolAddress) with
+ * that device current; make that first call before any stream capture.  All calls on a device
+ * share the one array and it keeps the last call's contents (the status word is cleared by each
+ * call), so calls whose kernels overlap on the GPU -- on different streams, or from different host
+ * threads -- race on it: serialise them.  Device-detected faults land in that shared status word
+ * and are not reported separately; use gdn_chunk_fwd with a workspace to read them.
+ */
+#define GDN_NOALLOC_SCRATCH_BYTES (64 * 1024)
+gdn_status gdn_chunk_fwd_noalloc(const void* q, const void* k, const void* v, const float* g,
+                                 const float* beta, gdn_dtype dtype, float scale,
+                                 const float* initial_state, const int32_t* cu_seqlens, int N,
+                                 int B, int64_t T, int Hk, int Hv, int dk, int dv, int chunk,
+                                 void* out, float* final_state, void* stream);
+
 /* Bytes of workspace gdn_chunk_fwd needs for these sizes (always > 0, a multiple of 256). */
 size_t gdn_chunk_fwd_workspace_size(int N, int B, int64_t T, int Hk, int Hv, int dk, int dv,
                                     int chunk);
