@@ -147,7 +147,11 @@ gdn_status gdn_chunk_fwd(const void* q, const void* k, const void* v, const floa
   int* status = reinterpret_cast<int*>(workspace);
   if (cudaMemsetAsync(status, 0, sizeof(int), s) != cudaSuccess) return GDN_ERR_CUDA;
   cudaError_t e;
-  e = launch_chunk_simt(q, k, v, g, beta, dtype, scale, initial_state, cu_seqlens, N, B, T, Hk,
+  if (dtype == GDN_BF16 && dk == 128 && dv == 128 && chunk == 64)
+    e = launch_chunk_tc(q, k, v, g, beta, scale, initial_state, cu_seqlens, N, B, T, Hk, Hv, out,
+                        final_state, status, s);
+  else
+    e = launch_chunk_simt(q, k, v, g, beta, dtype, scale, initial_state, cu_seqlens, N, B, T, Hk,
                           Hv, dk, dv, chunk, out, final_state, status, s);
   return from_cuda(e);
 }

@@ -51,7 +51,7 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, 10000;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
       : "r"(smem_u32(bar)), "r"(parity)
@@ -59,10 +59,22 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Waits for the phase with the given parity to complete.  Returns false if it never did.
+__device__ __forceinline__ uint64_t globaltimer_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+// Waits for the phase with the given parity to complete.  Gives up (returns false) after
+// kWaitLimitNs of wall-clock time or kSpinLimit polls, whichever comes first.
+constexpr uint64_t kWaitLimitNs = 4000000000ull;  // 4 s: every legitimate wait is microseconds
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
-  for (uint32_t i = 0; i < kSpinLimit; ++i)
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  for (uint32_t i = 0; i < kSpinLimit; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
+    if ((i & 63) == 63 && globaltimer_ns() - t0 > kWaitLimitNs) return false;
+  }
   return false;
 }
 
@@ -187,6 +199,37 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
 
 __device__ __forceinline__ void tmem_ld_wait() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+// 64 consecutive columns of this warp's 32 lanes (four x16 loads, one wait).
+__device__ __forceinline__ void tmem_ld64(uint32_t taddr, float (&v)[64]) {
+  float* p = v;
+  tmem_ld16(taddr + 0, *reinterpret_cast<float(*)[16]>(p + 0));
+  tmem_ld16(taddr + 16, *reinterpret_cast<float(*)[16]>(p + 16));
+  tmem_ld16(taddr + 32, *reinterpret_cast<float(*)[16]>(p + 32));
+  tmem_ld16(taddr + 48, *reinterpret_cast<float(*)[16]>(p + 48));
+  tmem_ld_wait();
+}
+
+// 32 consecutive columns (two x16 loads, one wait).
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
+  float* p = v;
+  tmem_ld16(taddr + 0, *reinterpret_cast<float(*)[16]>(p + 0));
+  tmem_ld16(taddr + 16, *reinterpret_cast<float(*)[16]>(p + 16));
+  tmem_ld_wait();
+}
+
+// Named barrier over `count` threads (a multiple of 32).
+__device__ __forceinline__ void named_bar(int id, int count) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
+// Byte offset of element (row, col) of a [rows][64] 2-byte tile stored with the 128-byte swizzle
+// (8-row atoms of 128-byte rows; the 16-byte chunk index is XORed with row % 8).  This is the
+// layout TMA writes with CU_TENSOR_MAP_SWIZZLE_128B and the tcgen05 descriptors read.
+__host__ __device__ __forceinline__ uint32_t sw128(int row, int col) {
+  return (uint32_t)row * 128u + ((((uint32_t)col >> 3) ^ ((uint32_t)row & 7u)) << 4) +
+         ((uint32_t)col & 7u) * 2u;
 }
 
 // ------------------------------------------------------------------ descriptors ------------

@@ -28,7 +28,7 @@ __device__ __forceinline__ float warp_sum(float x) {
 }
 
 template <typename T>
-__global__ void __launch_bounds__(REC_THREADS) recurrent_step_kernel(
+__global__ void __launch_bounds__(REC_THREADS, 3) recurrent_step_kernel(
     const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
     const float* __restrict__ g, const float* __restrict__ beta, float scale,
     float* __restrict__ state, int Hk, int Hv, int dv, T* __restrict__ out) {
@@ -48,38 +48,29 @@ __global__ void __launch_bounds__(REC_THREADS) recurrent_step_kernel(
   const T* vrow = v + (int64_t)nh * dv;
   T* orow = out + (int64_t)nh * dv;
 
+  // dv is a multiple of REC_ROWS (checked on the host), so a batch is either fully in range or
+  // not started.
   for (int base = warp * REC_ROWS; base < dv; base += (REC_THREADS / 32) * REC_ROWS) {
+    const float* Sb = S + (size_t)base * DK;
     float4 s[REC_ROWS];
 #pragma unroll
-    for (int u = 0; u < REC_ROWS; ++u)
-      if (base + u < dv) s[u] = __ldcs(reinterpret_cast<const float4*>(S + (int64_t)(base + u) * DK) + lane);
+    for (int u = 0; u < REC_ROWS; ++u) s[u] = __ldcs(reinterpret_cast<const float4*>(Sb + u * DK) + lane);
     float sk[REC_ROWS], sq[REC_ROWS];
 #pragma unroll
     for (int u = 0; u < REC_ROWS; ++u) {
-      if (base + u < dv) {
-        sk[u] = s[u].x * k4[0] + s[u].y * k4[1] + s[u].z * k4[2] + s[u].w * k4[3];
-        sq[u] = s[u].x * q4[0] + s[u].y * q4[1] + s[u].z * q4[2] + s[u].w * q4[3];
-      } else {
-        sk[u] = 0.0f;
-        sq[u] = 0.0f;
-      }
-    }
-#pragma unroll
-    for (int u = 0; u < REC_ROWS; ++u) {
-      sk[u] = warp_sum(sk[u]);
-      sq[u] = warp_sum(sq[u]);
+      sk[u] = warp_sum(s[u].x * k4[0] + s[u].y * k4[1] + s[u].z * k4[2] + s[u].w * k4[3]);
+      sq[u] = warp_sum(s[u].x * q4[0] + s[u].y * q4[1] + s[u].z * q4[2] + s[u].w * q4[3]);
     }
 #pragma unroll
     for (int u = 0; u < REC_ROWS; ++u) {
       const int j = base + u;
-      if (j >= dv) break;
       const float uj = b * (to_f(vrow[j]) - a * sk[u]);
       float4 o4;
       o4.x = fmaf(a, s[u].x, uj * k4[0]);
       o4.y = fmaf(a, s[u].y, uj * k4[1]);
       o4.z = fmaf(a, s[u].z, uj * k4[2]);
       o4.w = fmaf(a, s[u].w, uj * k4[3]);
-      __stcs(reinterpret_cast<float4*>(S + (int64_t)j * DK) + lane, o4);
+      __stcs(reinterpret_cast<float4*>(S + (size_t)j * DK) + lane, o4);
       if (lane == u) orow[j] = from_f<T>(scale * fmaf(a, sq[u], uj * kq));
     }
   }
