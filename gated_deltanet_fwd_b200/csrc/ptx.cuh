@@ -219,6 +219,77 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
   tmem_ld_wait();
 }
 
+// ------------------------------------------------------------------ warp-level tf32 MMA ----
+// mma.sync m16n8k8 with tf32 inputs and fp32 accumulation (used only for the small 16 x 16 block
+// products of the in-chunk triangular inverse).  Fragment ownership, with g = lane / 4 and
+// t = lane % 4:  A (16 x 8, row-major) a0 (g, t), a1 (g+8, t), a2 (g, t+4), a3 (g+8, t+4);
+// B (8 x 8, k x n) b0 (t, g), b1 (t+4, g);  C (16 x 8) c0 (g, 2t), c1 (g, 2t+1), c2 (g+8, 2t),
+// c3 (g+8, 2t+1).
+__device__ __forceinline__ uint32_t to_tf32(float x) {
+  uint32_t r;
+  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+  return r;
+}
+
+__device__ __forceinline__ void mma_tf32_16x8x8(float (&c)[4], uint32_t a0, uint32_t a1,
+                                                uint32_t a2, uint32_t a3, uint32_t b0,
+                                                uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// C (16 x 16, two n-tiles of 8) += X (16 x 16) * Y (16 x 16); X and Y are fp32 in shared memory
+// with row strides xs and ys (floats).  One warp.
+__device__ __forceinline__ void warp_mm16(const float* X, int xs, const float* Y, int ys,
+                                          float (&c)[2][4], int lane) {
+  const int g = lane >> 2, t = lane & 3;
+#pragma unroll
+  for (int kk = 0; kk < 2; ++kk) {
+    const uint32_t a0 = to_tf32(X[g * xs + 8 * kk + t]);
+    const uint32_t a1 = to_tf32(X[(g + 8) * xs + 8 * kk + t]);
+    const uint32_t a2 = to_tf32(X[g * xs + 8 * kk + t + 4]);
+    const uint32_t a3 = to_tf32(X[(g + 8) * xs + 8 * kk + t + 4]);
+#pragma unroll
+    for (int nn = 0; nn < 2; ++nn) {
+      const uint32_t b0 = to_tf32(Y[(8 * kk + t) * ys + 8 * nn + g]);
+      const uint32_t b1 = to_tf32(Y[(8 * kk + t + 4) * ys + 8 * nn + g]);
+      mma_tf32_16x8x8(c[nn], a0, a1, a2, a3, b0, b1);
+    }
+  }
+}
+
+// Stores sign * C (a warp_mm16 result) to a 16 x 16 fp32 block with row stride cs.
+__device__ __forceinline__ void warp_store16(float* C, int cs, const float (&c)[2][4], float sign,
+                                             int lane) {
+  const int g = lane >> 2, t = lane & 3;
+#pragma unroll
+  for (int nn = 0; nn < 2; ++nn) {
+    C[g * cs + 8 * nn + 2 * t] = sign * c[nn][0];
+    C[g * cs + 8 * nn + 2 * t + 1] = sign * c[nn][1];
+    C[(g + 8) * cs + 8 * nn + 2 * t] = sign * c[nn][2];
+    C[(g + 8) * cs + 8 * nn + 2 * t + 1] = sign * c[nn][3];
+  }
+}
+
+// Named barrier over `count` threads that also ANDs `ok` across them: every participant gets the
+// same answer, so a failure seen by one thread makes the whole group leave together (a group that
+// split up at a barrier would wait forever).
+__device__ __forceinline__ bool named_bar_and(int id, int count, bool ok) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 q, %3, 0;\n\t"
+      "bar.red.and.pred p, %1, %2, q;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(r)
+      : "r"(id), "r"(count), "r"((uint32_t)ok)
+      : "memory");
+  return r != 0;
+}
+
 // Named barrier over `count` threads (a multiple of 32).
 __device__ __forceinline__ void named_bar(int id, int count) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
