@@ -319,14 +319,11 @@ def bench_layer_core(dist, gdn, K, W, peaks):
     S_T = torch.empty(B, Hv, d, d, device=dev)
     cs_out = torch.empty(B, C, w["K"] - 1, device=dev)
     ws = torch.empty(gdn.workspace_size(B, B, T, Hk, Hv, d, d, 64), dtype=torch.uint8, device=dev)
-    # q, k, v are strided views into the conv output; the chunk call takes dense tensors, so the
-    # conv writes into one buffer laid out [q | k | v] per token and the views are made dense by
-    # running the conv on the mix and then splitting with a copy-free layout: the chunk kernel
-    # reads q at row stride C.  Until strided inputs are supported the split is a copy.
+    # q, k, v are views into the conv output [q | k | v] (token stride C): no copies
     kt = {"conv": KernelTimer(), "chunk": KernelTimer(), "norm": KernelTimer()}
-    qd = torch.empty(B, T, Hk, d, dtype=torch.bfloat16, device=dev)
-    kd = torch.empty_like(qd)
-    vd = torch.empty(B, T, Hv, d, dtype=torch.bfloat16, device=dev)
+    qv = y[:, :, :Hk * d].view(B, T, Hk, d)
+    kv = y[:, :, Hk * d:2 * Hk * d].view(B, T, Hk, d)
+    vv = y[:, :, 2 * Hk * d:].view(B, T, Hv, d)
     yout = torch.empty_like(core)
 
     def step(timed):
@@ -334,11 +331,8 @@ def bench_layer_core(dist, gdn, K, W, peaks):
         run("conv", lambda: gdn.gdn_causal_conv1d_silu(mix, conv_w, None, n_l2norm_ch=2 * Hk * d,
                                                        l2norm_group=d, conv_state_out=cs_out,
                                                        y=y))
-        qd.copy_(y[:, :, :Hk * d].view(B, T, Hk, d))
-        kd.copy_(y[:, :, Hk * d:2 * Hk * d].view(B, T, Hk, d))
-        vd.copy_(y[:, :, 2 * Hk * d:].view(B, T, Hv, d))
         gdn.gdn_gates(a, b, A_log, dt_bias, g=g, beta=beta)
-        run("chunk", lambda: gdn.gdn_chunk_fwd(qd, kd, vd, g, beta, scale=d ** -0.5, chunk=64,
+        run("chunk", lambda: gdn.gdn_chunk_fwd(qv, kv, vv, g, beta, scale=d ** -0.5, chunk=64,
                                                out=core, final_state=S_T, workspace=ws))
         run("norm", lambda: gdn.gdn_gated_rmsnorm(core, z, norm_w, eps=w["eps"], y=yout))
 

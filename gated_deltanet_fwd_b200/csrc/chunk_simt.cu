@@ -25,7 +25,7 @@ constexpr int SIMT_DVS = 64;  // value rows per block
 
 template <typename T>
 __global__ void __launch_bounds__(SIMT_THREADS) chunk_simt_kernel(
-    const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
+    const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v, TokStrides ts,
     const float* __restrict__ g, const float* __restrict__ beta, float scale,
     const float* __restrict__ S0, const int32_t* __restrict__ cu, int N, int64_t Tlen, int Hk,
     int Hv, int dk, int dv, int C, T* __restrict__ out, float* __restrict__ S_T,
@@ -78,13 +78,12 @@ __global__ void __launch_bounds__(SIMT_THREADS) chunk_simt_kernel(
     // ---- load the chunk
     for (int e = tid; e < L * dk; e += SIMT_THREADS) {
       const int r = e / dk, i = e - r * dk;
-      const int64_t off = ((c_beg + r) * Hk + hk) * dk + i;
-      Ks[r * dkp + i] = to_f(k[off]);
-      Qs[r * dkp + i] = to_f(q[off]);
+      Ks[r * dkp + i] = to_f(k[(c_beg + r) * ts.k + hk * dk + i]);
+      Qs[r * dkp + i] = to_f(q[(c_beg + r) * ts.q + hk * dk + i]);
     }
     for (int e = tid; e < L * DVS; e += SIMT_THREADS) {
       const int r = e / DVS, j = e - r * DVS;
-      Vs[r * dvp + j] = to_f(v[((c_beg + r) * Hv + h) * dv + j0 + j]);
+      Vs[r * dvp + j] = to_f(v[(c_beg + r) * ts.v + h * dv + j0 + j]);
     }
     if (tid == 0) {
       float acc = 0.0f;
@@ -178,7 +177,8 @@ static size_t simt_smem_bytes(int dk, int C) {
   return f * sizeof(float);
 }
 
-cudaError_t launch_chunk_simt(const void* q, const void* k, const void* v, const float* g,
+cudaError_t launch_chunk_simt(const void* q, const void* k, const void* v, TokStrides ts,
+                              const float* g,
                               const float* beta, gdn_dtype dt, float scale, const float* S0,
                               const int32_t* cu, int N, int B, int64_t T, int Hk, int Hv, int dk,
                               int dv, int chunk, void* out, float* S_T, int* status,
@@ -194,14 +194,14 @@ cudaError_t launch_chunk_simt(const void* q, const void* k, const void* v, const
                              cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     chunk_simt_kernel<__nv_bfloat16><<<(unsigned)blocks, SIMT_THREADS, smem, s>>>(
-        (const __nv_bfloat16*)q, (const __nv_bfloat16*)k, (const __nv_bfloat16*)v, g, beta, scale,
+        (const __nv_bfloat16*)q, (const __nv_bfloat16*)k, (const __nv_bfloat16*)v, ts, g, beta, scale,
         S0, cu, N, T, Hk, Hv, dk, dv, chunk, (__nv_bfloat16*)out, S_T, status);
   } else {
     e = cudaFuncSetAttribute(chunk_simt_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)smem);
     if (e != cudaSuccess) return e;
     chunk_simt_kernel<float><<<(unsigned)blocks, SIMT_THREADS, smem, s>>>(
-        (const float*)q, (const float*)k, (const float*)v, g, beta, scale, S0, cu, N, T, Hk, Hv,
+        (const float*)q, (const float*)k, (const float*)v, ts, g, beta, scale, S0, cu, N, T, Hk, Hv,
         dk, dv, chunk, (float*)out, S_T, status);
   }
   return cudaGetLastError();

@@ -17,18 +17,22 @@
 // One CTA per (sequence, v-head); the chunks of that chain run in order.  All five contractions are
 // M = 128 tcgen05 MMAs with 128-byte-swizzled shared-memory operands:
 //   D1  = [K; Q] K^T          (128 x 64,  K-dim 128)   -> K K^T and Q K^T for the prep warps
-//   DKS = [K; Gamma Q] S0^T   (128 x 128, K-dim 128)   -> K S0^T (for X) and Gamma Q S0^T
+//   DKS = [K; Q] S0^T         (128 x 128, K-dim 128)   -> K S0^T (for X) and Q S0^T (for O)
 //   DU  = [T'; P] X           (128 x 128, K-dim 64)    -> U in rows 0..63
-//   DKS += [T'; P] U          (accumulate)             -> rows 64..127 become Gamma Q S0^T + P U = O
-//   DS  = K'^T U              (128 x 128, K-dim 64)    -> the state increment (K' = decayed K)
+//   DU  = [T'; P] U           (after U is copied out)  -> P U in rows 64..127
+//   DS += K^T (D U)           (128 x 128, K-dim 64)    -> onto the decayed fp32 state, D = diag(e^{gamma_L - gamma})
+// and O = scale (Gamma_r (Q S0^T)_r + (P U)_r) is formed in the output epilogue.  The fp32 state S^T
+// lives in tensor memory: at the start of each chunk it is scaled by Gamma_L in place (while the
+// first MMA runs) and the last MMA accumulates the chunk's increment onto it; its bf16 copy in
+// shared memory is the next chunk's operand.
 // Warp roles (512 threads):
 //   warp 0      TMA producer: K, Q, V tiles of each chunk into a two-stage ring
-//   warps 4-7   prep, running ahead of the state chain: issue D1, build the decay vectors, A (fp32)
-//               and P, scale Q by Gamma in place, invert I + A (fp32 forward substitution on the
-//               16 x 16 diagonal blocks, tf32 mma.sync for the off-diagonal block products), write T'
-//   warps 8-15  state chain: hold S^T in fp32 registers (row i of S^T, 64 columns per thread),
-//               issue the four chain MMAs from one elected thread, build X, convert U, decay K
-//               into K', write O, update S and its bf16 operand copy.  Inside the chain the only
+//   warps 4-7   prep, running ahead of the state chain: issue D1, cumulative log-decays and write
+//               strengths, the decay masks of A (fp32) and P, invert I + A
+//               (fp32 forward substitution on the 16 x 16 diagonal blocks, tf32 mma.sync for the
+//               off-diagonal block products), write T'
+//   warps 8-15  state chain: issue the four chain MMAs from one elected thread, build X, convert U
+//               (plain and decayed), write O, refresh the bf16 state operand.  Inside the chain the only
 //               synchronisation is named barriers and waits on the chain's own MMA commits.
 // Every mbarrier wait is bounded; a wait that runs out records GDN_ERR_TIMEOUT and the CTA winds
 // down.
@@ -58,9 +62,7 @@ constexpr uint32_t TP_BUF = 16384;
 constexpr uint32_t OFF_AF = 180224;                    // fp32 A [64][AS]
 constexpr uint32_t OFF_TF = OFF_AF + 64 * AS * 4;      // fp32 T [64][AS]
 constexpr uint32_t OFF_MB = OFF_TF + 64 * AS * 4;      // fp32 4 x [16][MS] block products
-constexpr uint32_t OFF_DEC = OFF_MB + 4 * 16 * MS * 4; // 2 x {Gamma[64], Dec[64], GammaL, pad}
-constexpr uint32_t DEC_BUF = 132 * 4;
-constexpr uint32_t OFF_PV = OFF_DEC + 2 * DEC_BUF;     // prep: gamma*log2(e)[64], beta[64]
+constexpr uint32_t OFF_PV = OFF_MB + 4 * 16 * MS * 4;  // prep: a_t = e^{g_t}[64], beta[64]
 constexpr uint32_t OFF_BAR = OFF_PV + 2 * 64 * 4;      // mbarriers
 constexpr uint32_t N_BARS = 16;
 constexpr uint32_t SMEM_USED = OFF_BAR + N_BARS * 8 + 16;
@@ -76,6 +78,36 @@ enum {
 };
 static_assert(B_COUNT <= (int)N_BARS, "barrier space");
 
+// Optional phase timing, compiled in only with -DGDN_TC_TRACE: per-role clock64 accumulators of
+// CTA 0, written to TcParams::trace (8 slots per role) when the role finishes.
+#ifdef GDN_TC_TRACE
+#define TC_TRACE_DECL(active)                        \
+  const bool tr_on_ = (active) && blockIdx.x == 0; \
+  unsigned long long tr_acc_[8] = {};               \
+  unsigned long long tr_last_ = clock64();
+#define TC_TS(k)                                     \
+  do {                                               \
+    if (tr_on_) {                                    \
+      const unsigned long long n_ = clock64();       \
+      tr_acc_[k] += n_ - tr_last_;                   \
+      tr_last_ = n_;                                 \
+    }                                                \
+  } while (0)
+#define TC_TRACE_FLUSH(role)                                                    \
+  do {                                                                          \
+    if (tr_on_ && P.trace)                                                      \
+      for (int k_ = 0; k_ < 8; ++k_) P.trace[(role) * 8 + k_] = tr_acc_[k_];   \
+  } while (0)
+#else
+#define TC_TRACE_DECL(active)
+#define TC_TS(k) \
+  do {           \
+  } while (0)
+#define TC_TRACE_FLUSH(role) \
+  do {                       \
+  } while (0)
+#endif
+
 constexpr float kLog2e = 1.4426950408889634f;
 
 struct TcParams {
@@ -86,6 +118,7 @@ struct TcParams {
   __nv_bfloat16* out;
   float* S_T;
   int* status;
+  unsigned long long* trace;  // phase timing (trace builds only), else unused
   float scale;
   int N, Hk, Hv;
   int64_t T;
@@ -149,8 +182,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1) chunk_tc_kernel(
   if (tid == 0) {
     mbar_init(&bars[B_FULL0], 1);
     mbar_init(&bars[B_FULL1], 1);
-    mbar_init(&bars[B_EMPTY0], 3);  // chain MMAs done + prep done + chain read V
-    mbar_init(&bars[B_EMPTY1], 3);
+    mbar_init(&bars[B_EMPTY0], 2);  // chain MMAs (last: step 5) done + prep done
+    mbar_init(&bars[B_EMPTY1], 2);
     mbar_init(&bars[B_D1_FULL], 1);
     mbar_init(&bars[B_PREP_FULL0], 1);
     mbar_init(&bars[B_PREP_FULL1], 1);
@@ -212,17 +245,26 @@ __global__ void __launch_bounds__(TC_THREADS, 1) chunk_tc_kernel(
     float* Af = reinterpret_cast<float*>(smem + OFF_AF);
     float* Tf = reinterpret_cast<float*>(smem + OFF_TF);
     float* Mb = reinterpret_cast<float*>(smem + OFF_MB);
-    float* gl2 = reinterpret_cast<float*>(smem + OFF_PV);  // gamma * log2(e)
+    float* gl2 = reinterpret_cast<float*>(smem + OFF_PV);  // gamma * log2(e) of the chunk
     float* bet = gl2 + 64;
     const uint32_t id_d1 = idesc_bf16(128, 64, 0, 0);
+    // gates of the next chunk are fetched one chunk ahead (prep warp 0, rows lane and 32 + lane)
+    float pf_g0 = 0.0f, pf_g1 = 0.0f, pf_b0 = 0.0f, pf_b1 = 0.0f;
+    auto fetch_gates = [&](int c) {
+      const int64_t tc = s_beg + 64 * c;
+      const int Lc = (int)min((int64_t)64, s_end - tc);
+      pf_g0 = lane < Lc ? __ldg(P.g + (tc + lane) * P.Hv + h) : 0.0f;
+      pf_g1 = 32 + lane < Lc ? __ldg(P.g + (tc + 32 + lane) * P.Hv + h) : 0.0f;
+      pf_b0 = lane < Lc ? __ldg(P.beta + (tc + lane) * P.Hv + h) : 0.0f;
+      pf_b1 = 32 + lane < Lc ? __ldg(P.beta + (tc + 32 + lane) * P.Hv + h) : 0.0f;
+    };
+    if (pw == 0 && nchunks > 0) fetch_gates(0);
+    TC_TRACE_DECL(leader);
     for (int c = 0; c < nchunks; ++c) {
       const int st = c & 1, b = c & 1;
-      const int64_t t0 = s_beg + 64 * c;
-      const int L = (int)min((int64_t)64, s_end - t0);
-      unsigned char* kq = smem + OFF_KQ + st * KQ_STAGE;
       unsigned char* tp = smem + OFF_TP + b * TP_BUF;
-      float* dec = reinterpret_cast<float*>(smem + OFF_DEC + b * DEC_BUF);
       bool ok = true;
+      TC_TS(7);
       // D1 = [K; Q] K^T as soon as the chunk has landed (prep owns D1's tensor memory)
       if (leader) {
         ok = mbar_wait(&bars[B_FULL0 + st], (c >> 1) & 1);
@@ -237,12 +279,10 @@ __global__ void __launch_bounds__(TC_THREADS, 1) chunk_tc_kernel(
           mma_commit(&bars[B_D1_FULL]);
         }
       }
-      // decay vectors while D1 runs (warp 0 of prep); rows >= L carry zero decay, zero beta
+      // per-token decays and write strengths while D1 runs; rows past the sequence end carry
+      // zero log-decay (a_t = 1) and zero beta, which makes their corrections exactly zero
       if (pw == 0) {
-        float x0 = lane < L ? __ldg(P.g + (t0 + lane) * P.Hv + h) : 0.0f;
-        float x1 = 32 + lane < L ? __ldg(P.g + (t0 + 32 + lane) * P.Hv + h) : 0.0f;
-        const float b0 = lane < L ? __ldg(P.beta + (t0 + lane) * P.Hv + h) : 0.0f;
-        const float b1 = 32 + lane < L ? __ldg(P.beta + (t0 + 32 + lane) * P.Hv + h) : 0.0f;
+        float x0 = pf_g0, x1 = pf_g1;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
           const float y0 = __shfl_up_sync(0xffffffffu, x0, o);
@@ -253,19 +293,13 @@ __global__ void __launch_bounds__(TC_THREADS, 1) chunk_tc_kernel(
           }
         }
         x1 += __shfl_sync(0xffffffffu, x0, 31);
-        const float glast = __shfl_sync(0xffffffffu, x1, 31);
         gl2[lane] = x0 * kLog2e;
         gl2[32 + lane] = x1 * kLog2e;
-        bet[lane] = b0;
-        bet[32 + lane] = b1;
-        // the chain's copy (buffer b) is free: the chain read it at the start of chunk c - 2,
-        // before it issued the MMAs whose completion prep_empty[b] (waited below) reports
-        dec[lane] = __expf(x0);
-        dec[32 + lane] = __expf(x1);
-        dec[64 + lane] = __expf(glast - x0);
-        dec[96 + lane] = __expf(glast - x1);
-        if (lane == 0) dec[128] = __expf(glast);
+        bet[lane] = pf_b0;
+        bet[32 + lane] = pf_b1;
+        if (c + 1 < nchunks) fetch_gates(c + 1);
       }
+      TC_TS(0);
       ok = ok && mbar_wait(&bars[B_PREP_EMPTY0 + b], ((c >> 1) & 1) ^ 1) &&
            mbar_wait(&bars[B_D1_FULL], c & 1);
       // one decision for all prep threads; also makes gl2 / bet visible to them
@@ -273,57 +307,51 @@ __global__ void __launch_bounds__(TC_THREADS, 1) chunk_tc_kernel(
         fail(GDN_ERR_TIMEOUT);
         break;
       }
+      TC_TS(1);
       tc_fence_after();
       {
         // this thread's row of D1: rows 0..63 are K K^T, rows 64..127 are Q K^T
-        float d[64];
-        tmem_ld64(tmem + TM_D1 + ((uint32_t)(32 * pw) << 16), d);
-        if (pw < 2) {
-          const int r = 32 * pw + lane;
-          const float gr = gl2[r], br = bet[r];
-          float* arow = Af + r * AS;
+        // e^{gamma_r - gamma_s} = 2^{(gamma_r - gamma_s) log2 e}: only differences of in-chunk
+        // cumulative log-decays are exponentiated (s <= r, so never above 1).  Each 32-column half
+        // is loaded in full (tensor memory and shared memory) before anything is stored.
+        const int r = 32 * (pw & 1) + lane;
+        const float gr = gl2[r];
+        const float br = pw < 2 ? bet[r] : 1.0f;
+        float* arow = Af + r * AS;
 #pragma unroll
-          for (int s4 = 0; s4 < 16; ++s4) {
-            const float4 gs = *reinterpret_cast<const float4*>(gl2 + 4 * s4);
-            float4 a4;
-            a4.x = (4 * s4 + 0 < r) ? br * ex2(gr - gs.x) * d[4 * s4 + 0] : 0.0f;
-            a4.y = (4 * s4 + 1 < r) ? br * ex2(gr - gs.y) * d[4 * s4 + 1] : 0.0f;
-            a4.z = (4 * s4 + 2 < r) ? br * ex2(gr - gs.z) * d[4 * s4 + 2] : 0.0f;
-            a4.w = (4 * s4 + 3 < r) ? br * ex2(gr - gs.w) * d[4 * s4 + 3] : 0.0f;
-            *reinterpret_cast<float4*>(arow + 4 * s4) = a4;
+        for (int half = 0; half < 2; ++half) {
+          float d[32], gs[32];
+          tmem_ld16(tmem + TM_D1 + ((uint32_t)(32 * pw) << 16) + 32 * half,
+                    *reinterpret_cast<float(*)[16]>(d));
+          tmem_ld16(tmem + TM_D1 + ((uint32_t)(32 * pw) << 16) + 32 * half + 16,
+                    *reinterpret_cast<float(*)[16]>(d + 16));
+#pragma unroll
+          for (int q4 = 0; q4 < 8; ++q4)
+            *reinterpret_cast<float4*>(gs + 4 * q4) =
+                *reinterpret_cast<const float4*>(gl2 + 32 * half + 4 * q4);
+          tmem_ld_wait();
+          float v[32];
+#pragma unroll
+          for (int q = 0; q < 32; ++q) {
+            const int sidx = 32 * half + q;
+            const bool keep = pw < 2 ? (sidx < r) : (sidx <= r);
+            v[q] = keep ? br * ex2(gr - gs[q]) * d[q] : 0.0f;
           }
-        } else {
-          const int r = 32 * (pw - 2) + lane;
-          const float gr = gl2[r];
+          if (pw < 2) {
 #pragma unroll
-          for (int s8 = 0; s8 < 8; ++s8) {
-            const float4 ga = *reinterpret_cast<const float4*>(gl2 + 8 * s8);
-            const float4 gb = *reinterpret_cast<const float4*>(gl2 + 8 * s8 + 4);
-            const float gsv[8] = {ga.x, ga.y, ga.z, ga.w, gb.x, gb.y, gb.z, gb.w};
-            float pv[8];
+            for (int q4 = 0; q4 < 8; ++q4)
+              *reinterpret_cast<float4*>(arow + 32 * half + 4 * q4) =
+                  make_float4(v[4 * q4], v[4 * q4 + 1], v[4 * q4 + 2], v[4 * q4 + 3]);
+          } else {
 #pragma unroll
-            for (int e = 0; e < 8; ++e)
-              pv[e] = (8 * s8 + e <= r) ? ex2(gr - gsv[e]) * d[8 * s8 + e] : 0.0f;
-            *reinterpret_cast<uint4*>(tp + sw128(64 + r, 8 * s8)) = pack8(pv);
+            for (int q8 = 0; q8 < 4; ++q8)
+              *reinterpret_cast<uint4*>(tp + sw128(64 + r, 32 * half + 8 * q8)) = pack8(&v[8 * q8]);
           }
         }
       }
-      // Gamma Q in place (D1 has consumed the unscaled Q)
-      {
-        const int r = p >> 1, hh = p & 1;
-        const float gq = ex2(gl2[r]);
-        unsigned char* qrow = kq + hh * 16384 + 8192;
-#pragma unroll
-        for (int c8 = 0; c8 < 8; ++c8) {
-          uint4* ptr = reinterpret_cast<uint4*>(qrow + sw128(r, 8 * c8));
-          float f[8];
-          unpack8(*ptr, f);
-#pragma unroll
-          for (int e = 0; e < 8; ++e) f[e] *= gq;
-          *ptr = pack8(f);
-        }
-      }
+      TC_TS(2);
       named_bar(1, 128);  // A complete
+      TC_TS(3);
       // ---- T = (I + A)^{-1}.  Diagonal 16 x 16 blocks: fp32 forward substitution, one column
       // per lane, four partial sums per row.
       if (pw < 2) {
@@ -346,6 +374,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) chunk_tc_kernel(
         for (int r = 0; r < 16; ++r) Tf[(16 * blk + r) * AS + col] = x[r];
       }
       named_bar(1, 128);
+      TC_TS(4);
       // Off-diagonal blocks by distance:  T_ij = -T_ii sum_{k=j}^{i-1} A_ik T_kj.
       // Distance 1: warps 1..3 each own block (i, i-1).
       if (pw >= 1) {
@@ -404,25 +433,23 @@ __global__ void __launch_bounds__(TC_THREADS, 1) chunk_tc_kernel(
         warp_store16(Tf + 48 * AS + 0, AS, t2, -1.0f, lane);
       }
       named_bar(1, 128);
+      TC_TS(5);
       // T' = T diag(beta) -> rows 0..63 of the [T'; P] tile (bf16, K-major); zero above the
       // diagonal (the solve leaves that part of Tf unwritten)
       {
         const int r = p >> 1, s0 = 32 * (p & 1);
         const float* trow = Tf + r * AS;
+        float tv[32], bv[32];
 #pragma unroll
-        for (int c8 = 0; c8 < 4; ++c8) {
-          const int sb = s0 + 8 * c8;
-          const float4 t0v = *reinterpret_cast<const float4*>(trow + sb);
-          const float4 t1v = *reinterpret_cast<const float4*>(trow + sb + 4);
-          const float4 b0v = *reinterpret_cast<const float4*>(bet + sb);
-          const float4 b1v = *reinterpret_cast<const float4*>(bet + sb + 4);
-          float tv[8] = {t0v.x * b0v.x, t0v.y * b0v.y, t0v.z * b0v.z, t0v.w * b0v.w,
-                         t1v.x * b1v.x, t1v.y * b1v.y, t1v.z * b1v.z, t1v.w * b1v.w};
-#pragma unroll
-          for (int e = 0; e < 8; ++e)
-            if (sb + e > r) tv[e] = 0.0f;
-          *reinterpret_cast<uint4*>(tp + sw128(r, sb)) = pack8(tv);
+        for (int q4 = 0; q4 < 8; ++q4) {
+          *reinterpret_cast<float4*>(tv + 4 * q4) = *reinterpret_cast<const float4*>(trow + s0 + 4 * q4);
+          *reinterpret_cast<float4*>(bv + 4 * q4) = *reinterpret_cast<const float4*>(bet + s0 + 4 * q4);
         }
+#pragma unroll
+        for (int q = 0; q < 32; ++q) tv[q] = (s0 + q <= r) ? tv[q] * bv[q] : 0.0f;
+#pragma unroll
+        for (int c8 = 0; c8 < 4; ++c8)
+          *reinterpret_cast<uint4*>(tp + sw128(r, s0 + 8 * c8)) = pack8(&tv[8 * c8]);
       }
       fence_proxy_async_smem();
       tc_fence_before();
@@ -431,7 +458,9 @@ __global__ void __launch_bounds__(TC_THREADS, 1) chunk_tc_kernel(
         mbar_arrive(&bars[B_PREP_FULL0 + b]);
         mbar_arrive(&bars[B_EMPTY0 + st]);
       }
+      TC_TS(6);
     }
+    TC_TRACE_FLUSH(2);
     if (leader) {
       mma_commit(&bars[B_DRAIN_P]);
       mbar_wait(&bars[B_DRAIN_P], 0);
@@ -446,25 +475,35 @@ __global__ void __launch_bounds__(TC_THREADS, 1) chunk_tc_kernel(
     const uint32_t id_ks = idesc_bf16(128, 128, 0, 1);
     const uint32_t id_u = idesc_bf16(128, 128, 0, 1);
     const uint32_t id_s = idesc_bf16(128, 128, 1, 1);
-    float sreg[64];
+    // The fp32 state lives in tensor memory (TM_S: lane i = row of S^T, 128 value columns); this
+    // thread owns lane i, columns jb..jb+63.  Its bf16 copy in shared memory is step 1's operand.
     const size_t sbase_g = ((size_t)n * P.Hv + h) * 128 * 128;
-    if (P.S0) {
+    const uint32_t s_tm = tmem + TM_S + jb + lane_off;
+    unsigned char* sb = smem + OFF_SB + hf * 16384;
 #pragma unroll
-      for (int jj = 0; jj < 64; ++jj)
-        sreg[jj] = __ldg(P.S0 + sbase_g + (size_t)(jb + jj) * 128 + i);
-    } else {
+    for (int pc = 0; pc < 4; ++pc) {
+      float v16[16];
 #pragma unroll
-      for (int jj = 0; jj < 64; ++jj) sreg[jj] = 0.0f;
+      for (int jj = 0; jj < 16; ++jj)
+        v16[jj] = P.S0 ? __ldg(P.S0 + sbase_g + (size_t)(jb + 16 * pc + jj) * 128 + i) : 0.0f;
+      tmem_st16(s_tm + 16 * pc, v16);
+      *reinterpret_cast<uint4*>(sb + sw128(i, 16 * pc)) = pack8(&v16[0]);
+      *reinterpret_cast<uint4*>(sb + sw128(i, 16 * pc + 8)) = pack8(&v16[8]);
     }
-    auto write_sb = [&]() {
-      unsigned char* sb = smem + OFF_SB + hf * 16384;
-#pragma unroll
-      for (int c8 = 0; c8 < 8; ++c8)
-        *reinterpret_cast<uint4*>(sb + sw128(i, 8 * c8)) = pack8(&sreg[8 * c8]);
-      fence_proxy_async_smem();
-    };
-    write_sb();
+    tmem_st_wait();
+    fence_proxy_async_smem();
+    tc_fence_before();
     named_bar(2, 256);
+    // log-decays of the next chunk are fetched one chunk ahead (rows lane and 32 + lane)
+    float pg0 = 0.0f, pg1 = 0.0f;
+    auto fetch_g = [&](int c) {
+      const int64_t tc = s_beg + 64 * c;
+      const int Lc = (int)min((int64_t)64, s_end - tc);
+      pg0 = lane < Lc ? __ldg(P.g + (tc + lane) * P.Hv + h) : 0.0f;
+      pg1 = 32 + lane < Lc ? __ldg(P.g + (tc + 32 + lane) * P.Hv + h) : 0.0f;
+    };
+    if (nchunks > 0) fetch_g(0);
+    TC_TRACE_DECL(leader || e == 64);
 
     // Exits are decided jointly (named_bar_and): a wait that ran out in any thread makes all 256
     // leave at the same barrier.
@@ -477,14 +516,29 @@ __global__ void __launch_bounds__(TC_THREADS, 1) chunk_tc_kernel(
       const uint32_t tpa = sbase + OFF_TP + b * TP_BUF;
       unsigned char* kq = smem + OFF_KQ + st * KQ_STAGE;
       unsigned char* vt = smem + OFF_V + st * V_STAGE;
-      // prep for this chunk done (T', P, Gamma Q, decay vectors); the TMA data has landed
-      bool ok = mbar_wait(&bars[B_PREP_FULL0 + b], (c >> 1) & 1) &&
-                mbar_wait(&bars[B_FULL0 + st], (c >> 1) & 1);
-      const float* dec = reinterpret_cast<const float*>(smem + OFF_DEC + b * DEC_BUF);
-      const float g_row = dec[i & 63];          // Gamma_r for r = i (rows 0..63)
-      const float d_row = dec[64 + (i & 63)];   // e^{gamma_63 - gamma_s} for s = i - 64
-      const float gC = dec[128];
-      // step 1: D_KS = [K; Gamma Q] S0^T
+      TC_TS(7);
+      // in-chunk cumulative log-decay (inclusive scan over the chunk's 64 rows)
+      float gl = pg0, gh = pg1;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const float y0 = __shfl_up_sync(0xffffffffu, gl, o);
+        const float y1 = __shfl_up_sync(0xffffffffu, gh, o);
+        if (lane >= o) {
+          gl += y0;
+          gh += y1;
+        }
+      }
+      gh += __shfl_sync(0xffffffffu, gl, 31);
+      const float glast = __shfl_sync(0xffffffffu, gh, 31);
+      if (c + 1 < nchunks) fetch_g(c + 1);
+      // this thread's row r: i for rows 0..63, i - 64 for rows 64..127
+      const float g_row = __expf((ew & 1) ? gh : gl);           // Gamma_r
+      const float d_row = __expf(glast - ((ew & 1) ? gh : gl)); // e^{gamma_63 - gamma_r}
+      const float gC = __expf(glast);
+      // the chunk's K, Q, V have landed (step 1 needs nothing from the prep warps)
+      bool ok = mbar_wait(&bars[B_FULL0 + st], (c >> 1) & 1);
+      TC_TS(0);
+      // step 1: D_KS = [K; Q] S0^T
       if (leader && ok) {
         tc_fence_after();
         for (int ks = 0; ks < 8; ++ks) {
@@ -495,39 +549,42 @@ __global__ void __launch_bounds__(TC_THREADS, 1) chunk_tc_kernel(
         }
         mma_commit(&bars[B_M_KS]);
       }
+      // S <- Gamma_L S in tensor memory while step 1 runs (step 5 then accumulates K^T D U onto it;
+      // the previous chunk's step 5 has completed)
+#pragma unroll
+      for (int pc = 0; pc < 2; ++pc) {
+        float v[32];
+        tmem_ld32(s_tm + 32 * pc, v);
+#pragma unroll
+        for (int jj = 0; jj < 32; ++jj) v[jj] *= gC;
+        tmem_st16(s_tm + 32 * pc, *reinterpret_cast<float(*)[16]>(v));
+        tmem_st16(s_tm + 32 * pc + 16, *reinterpret_cast<float(*)[16]>(v + 16));
+      }
+      tmem_st_wait();
       ok = ok && mbar_wait(&bars[B_M_KS], par);
+      TC_TS(1);
       tc_fence_after();
       if (!ok) {
         // skip the work; the joint barrier below takes everyone out
       } else if (ew < 2) {
         // X = V - Gamma_r (K S0^T), rows r = i
         unsigned char* xu = smem + OFF_XU + hf * 8192;
+        float ks[64];
+        uint4 vraw[8];
 #pragma unroll
-        for (int pc = 0; pc < 2; ++pc) {
-          float ks[32];
-          tmem_ld32(tmem + TM_KS + jb + 32 * pc + lane_off, ks);
+        for (int q = 0; q < 4; ++q)
+          tmem_ld16(tmem + TM_KS + jb + 16 * q + lane_off, *reinterpret_cast<float(*)[16]>(ks + 16 * q));
 #pragma unroll
-          for (int c4 = 0; c4 < 4; ++c4) {
-            const int c8 = 4 * pc + c4;
-            float vf[8];
-            unpack8(*reinterpret_cast<const uint4*>(vt + hf * 8192 + sw128(i, 8 * c8)), vf);
-#pragma unroll
-            for (int q = 0; q < 8; ++q) vf[q] = fmaf(-g_row, ks[8 * c4 + q], vf[q]);
-            *reinterpret_cast<uint4*>(xu + sw128(i, 8 * c8)) = pack8(vf);
-          }
-        }
-      } else {
-        // K' = e^{gamma_63 - gamma_s} K in place, rows s = i - 64, dk half hf
-        const int s = i - 64;
-        unsigned char* krow = kq + hf * 16384;
+        for (int c8 = 0; c8 < 8; ++c8)
+          vraw[c8] = *reinterpret_cast<const uint4*>(vt + hf * 8192 + sw128(i, 8 * c8));
+        tmem_ld_wait();
 #pragma unroll
         for (int c8 = 0; c8 < 8; ++c8) {
-          uint4* ptr = reinterpret_cast<uint4*>(krow + sw128(s, 8 * c8));
-          float f[8];
-          unpack8(*ptr, f);
+          float vf[8];
+          unpack8(vraw[c8], vf);
 #pragma unroll
-          for (int q = 0; q < 8; ++q) f[q] *= d_row;
-          *ptr = pack8(f);
+          for (int q = 0; q < 8; ++q) vf[q] = fmaf(-g_row, ks[8 * c8 + q], vf[q]);
+          *reinterpret_cast<uint4*>(xu + sw128(i, 8 * c8)) = pack8(vf);
         }
       }
       fence_proxy_async_smem();
@@ -536,10 +593,12 @@ __global__ void __launch_bounds__(TC_THREADS, 1) chunk_tc_kernel(
         fail(GDN_ERR_TIMEOUT);
         break;
       }
-      // step 3: D_U = [T'; P] X
-      if (leader) {
+      TC_TS(2);
+      // step 3: D_U = [T'; P] X  (needs this chunk's T' and P from the prep warps; prep_full also
+      // means the prep's K K^T MMA has finished reading this stage's K)
+      ok = mbar_wait(&bars[B_PREP_FULL0 + b], (c >> 1) & 1);
+      if (leader && ok) {
         tc_fence_after();
-        mbar_arrive(&bars[B_EMPTY0 + st]);  // V of this stage consumed
         for (int ks = 0; ks < 4; ++ks) {
           const uint32_t a = tpa + (uint32_t)ks * 32u;
           const uint32_t bb = sbase + OFF_XU + (uint32_t)ks * 2048u;
@@ -548,11 +607,15 @@ __global__ void __launch_bounds__(TC_THREADS, 1) chunk_tc_kernel(
         }
         mma_commit(&bars[B_M_U]);
       }
-      ok = mbar_wait(&bars[B_M_U], par);
+      ok = ok && mbar_wait(&bars[B_M_U], par);
+      TC_TS(3);
       tc_fence_after();
       if (ok && ew < 2) {
-        // U rows 0..63 -> bf16 operand (overwrites X: the MMA that read X has completed)
+        // U rows 0..63 -> bf16 operands: U itself (for P U; overwrites X, whose MMA has
+        // completed) and e^{gamma_63 - gamma_s} U_s (for the state increment K^T diag(.) U; into
+        // this stage's V buffer, which X has consumed)
         unsigned char* xu = smem + OFF_XU + hf * 8192;
+        unsigned char* ud = vt + hf * 8192;
 #pragma unroll
         for (int pc = 0; pc < 2; ++pc) {
           float uv[32];
@@ -560,6 +623,11 @@ __global__ void __launch_bounds__(TC_THREADS, 1) chunk_tc_kernel(
 #pragma unroll
           for (int c4 = 0; c4 < 4; ++c4)
             *reinterpret_cast<uint4*>(xu + sw128(i, 8 * (4 * pc + c4))) = pack8(&uv[8 * c4]);
+#pragma unroll
+          for (int q = 0; q < 32; ++q) uv[q] *= d_row;
+#pragma unroll
+          for (int c4 = 0; c4 < 4; ++c4)
+            *reinterpret_cast<uint4*>(ud + sw128(i, 8 * (4 * pc + c4))) = pack8(&uv[8 * c4]);
         }
       }
       fence_proxy_async_smem();
@@ -568,40 +636,51 @@ __global__ void __launch_bounds__(TC_THREADS, 1) chunk_tc_kernel(
         fail(GDN_ERR_TIMEOUT);
         break;
       }
-      // steps 3b and 5: D_KS += [T'; P] U (rows 64..127 become O);  D_S = K'^T U
+      TC_TS(4);
+      // steps 3b and 5: D_U = [T'; P] U (rows 64..127 are P U; U itself is already in shared
+      // memory);  D_S += K^T (D U)
       if (leader) {
         tc_fence_after();
         for (int ks = 0; ks < 4; ++ks) {
           const uint32_t a = tpa + (uint32_t)ks * 32u;
           const uint32_t bb = sbase + OFF_XU + (uint32_t)ks * 2048u;
-          mma_bf16_ss(tmem + TM_KS, sdesc_sw128(a, 16, 1024), sdesc_sw128(bb, 8192, 1024), id_u,
-                      1);
+          mma_bf16_ss(tmem + TM_U, sdesc_sw128(a, 16, 1024), sdesc_sw128(bb, 8192, 1024), id_u,
+                      ks > 0);
         }
         for (int ks = 0; ks < 4; ++ks) {
           const uint32_t a = kqa + (uint32_t)ks * 2048u;
-          const uint32_t bb = sbase + OFF_XU + (uint32_t)ks * 2048u;
+          const uint32_t bb = sbase + OFF_V + st * V_STAGE + (uint32_t)ks * 2048u;
           mma_bf16_ss(tmem + TM_S, sdesc_sw128(a, 16384, 1024), sdesc_sw128(bb, 8192, 1024), id_s,
-                      ks > 0);
+                      1);
         }
         mma_commit(&bars[B_M_S]);
         mma_commit(&bars[B_PREP_EMPTY0 + b]);
         mma_commit(&bars[B_EMPTY0 + st]);
       }
       ok = mbar_wait(&bars[B_M_S], par);
+      TC_TS(5);
       tc_fence_after();
       if (ok && ew >= 2) {
         const int r = i - 64;
         __nv_bfloat16* orow = P.out + ((t0 + r) * P.Hv + h) * 128 + jb;
 #pragma unroll
         for (int pc = 0; pc < 2; ++pc) {
-          float o[32];
-          tmem_ld32(tmem + TM_KS + jb + 32 * pc + lane_off, o);
+          // O = scale (Gamma_r (Q S0^T)_r + (P U)_r)
+          float qs[32], pu[32];
+          tmem_ld16(tmem + TM_KS + jb + 32 * pc + lane_off, *reinterpret_cast<float(*)[16]>(qs));
+          tmem_ld16(tmem + TM_KS + jb + 32 * pc + 16 + lane_off,
+                    *reinterpret_cast<float(*)[16]>(qs + 16));
+          tmem_ld16(tmem + TM_U + jb + 32 * pc + lane_off, *reinterpret_cast<float(*)[16]>(pu));
+          tmem_ld16(tmem + TM_U + jb + 32 * pc + 16 + lane_off,
+                    *reinterpret_cast<float(*)[16]>(pu + 16));
+          tmem_ld_wait();
           if (r < L) {
 #pragma unroll
             for (int c4 = 0; c4 < 4; ++c4) {
               float f[8];
 #pragma unroll
-              for (int q = 0; q < 8; ++q) f[q] = P.scale * o[8 * c4 + q];
+              for (int q = 0; q < 8; ++q)
+                f[q] = P.scale * fmaf(g_row, qs[8 * c4 + q], pu[8 * c4 + q]);
               *reinterpret_cast<uint4*>(orow + 8 * (4 * pc + c4)) = pack8(f);
             }
           }
@@ -610,27 +689,34 @@ __global__ void __launch_bounds__(TC_THREADS, 1) chunk_tc_kernel(
       if (ok) {
 #pragma unroll
         for (int pc = 0; pc < 2; ++pc) {
-          float ds[32];
-          tmem_ld32(tmem + TM_S + jb + 32 * pc + lane_off, ds);
+          float sv[32];
+          tmem_ld32(s_tm + 32 * pc, sv);
 #pragma unroll
-          for (int jj = 0; jj < 32; ++jj)
-            sreg[32 * pc + jj] = fmaf(gC, sreg[32 * pc + jj], ds[jj]);
+          for (int c4 = 0; c4 < 4; ++c4)
+            *reinterpret_cast<uint4*>(sb + sw128(i, 32 * pc + 8 * c4)) = pack8(&sv[8 * c4]);
         }
-        write_sb();
+        fence_proxy_async_smem();
       }
       tc_fence_before();
       if (!named_bar_and(2, 256, ok)) {
         fail(GDN_ERR_TIMEOUT);
         break;
       }
+      TC_TS(6);
     }
+    TC_TRACE_FLUSH(leader ? 3 : 4);
     if (leader) {
       mma_commit(&bars[B_DRAIN_S]);
       mbar_wait(&bars[B_DRAIN_S], 0);
     }
     if (P.S_T && !*abort_flag) {
 #pragma unroll
-      for (int jj = 0; jj < 64; ++jj) P.S_T[sbase_g + (size_t)(jb + jj) * 128 + i] = sreg[jj];
+      for (int pc = 0; pc < 2; ++pc) {
+        float sv[32];
+        tmem_ld32(s_tm + 32 * pc, sv);
+#pragma unroll
+        for (int jj = 0; jj < 32; ++jj) P.S_T[sbase_g + (size_t)(jb + 32 * pc + jj) * 128 + i] = sv[jj];
+      }
     }
   }
 
@@ -663,12 +749,13 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// [rows, heads, 128] bf16 -> 3D map {128, heads, rows}, box {64, 1, 64}, 128-byte swizzle.
-bool make_map(CUtensorMap* m, const void* base, int heads, int64_t rows) {
+// [rows, heads, 128] bf16 with `tok_stride` elements between rows -> 3D map {128, heads, rows},
+// box {64, 1, 64}, 128-byte swizzle.
+bool make_map(CUtensorMap* m, const void* base, int heads, int64_t rows, int64_t tok_stride) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return false;
   cuuint64_t dims[3] = {128, (cuuint64_t)heads, (cuuint64_t)rows};
-  cuuint64_t strides[2] = {128 * 2, (cuuint64_t)heads * 128 * 2};
+  cuuint64_t strides[2] = {128 * 2, (cuuint64_t)tok_stride * 2};
   cuuint32_t box[3] = {64, 1, 64};
   cuuint32_t es[3] = {1, 1, 1};
   return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
@@ -678,18 +765,21 @@ bool make_map(CUtensorMap* m, const void* base, int heads, int64_t rows) {
 
 }  // namespace
 
-cudaError_t launch_chunk_tc(const void* q, const void* k, const void* v, const float* g,
-                            const float* beta, float scale, const float* S0, const int32_t* cu,
-                            int N, int B, int64_t T, int Hk, int Hv, void* out, float* S_T,
-                            int* status, cudaStream_t s) {
+namespace {
+cudaError_t launch_chunk_tc_impl(const void* q, const void* k, const void* v, TokStrides ts,
+                                 const float* g,
+                                 const float* beta, float scale, const float* S0,
+                                 const int32_t* cu, int N, int B, int64_t T, int Hk, int Hv,
+                                 void* out, float* S_T, int* status, unsigned long long* trace,
+                                 cudaStream_t s) {
   const int64_t rows = (int64_t)B * T;
   const int64_t ctas = (int64_t)N * Hv;
   if (ctas == 0) return cudaSuccess;
   if (ctas > 0x7fffffff) return cudaErrorInvalidConfiguration;
   CUtensorMap mq, mk, mv;
   const int64_t map_rows = rows > 0 ? rows : 1;
-  if (!make_map(&mq, q, Hk, map_rows) || !make_map(&mk, k, Hk, map_rows) ||
-      !make_map(&mv, v, Hv, map_rows))
+  if (!make_map(&mq, q, Hk, map_rows, ts.q) || !make_map(&mk, k, Hk, map_rows, ts.k) ||
+      !make_map(&mv, v, Hv, map_rows, ts.v))
     return cudaErrorInvalidValue;
   TcParams p;
   p.g = g;
@@ -699,6 +789,7 @@ cudaError_t launch_chunk_tc(const void* q, const void* k, const void* v, const f
   p.out = reinterpret_cast<__nv_bfloat16*>(out);
   p.S_T = S_T;
   p.status = status;
+  p.trace = trace;
   p.scale = scale;
   p.N = N;
   p.Hk = Hk;
@@ -710,6 +801,16 @@ cudaError_t launch_chunk_tc(const void* q, const void* k, const void* v, const f
   if (e != cudaSuccess) return e;
   chunk_tc_kernel<<<(unsigned)ctas, TC_THREADS, SMEM_BYTES, s>>>(mq, mk, mv, p);
   return cudaGetLastError();
+}
+}  // namespace
+
+cudaError_t launch_chunk_tc(const void* q, const void* k, const void* v, TokStrides ts,
+                            const float* g,
+                            const float* beta, float scale, const float* S0, const int32_t* cu,
+                            int N, int B, int64_t T, int Hk, int Hv, void* out, float* S_T,
+                            int* status, cudaStream_t s) {
+  return launch_chunk_tc_impl(q, k, v, ts, g, beta, scale, S0, cu, N, B, T, Hk, Hv, out, S_T, status,
+                              nullptr, s);
 }
 
 }  // namespace gdn

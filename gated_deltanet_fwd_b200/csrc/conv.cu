@@ -31,7 +31,7 @@ __device__ __forceinline__ void seq_range(const int32_t* cu, int64_t T, int n, i
 }
 
 template <typename T, int K>
-__global__ void __launch_bounds__(CONV_THREADS) conv_silu_kernel(
+__global__ void __launch_bounds__(CONV_THREADS, 4) conv_silu_kernel(
     const T* __restrict__ x, const float* __restrict__ w, const float* __restrict__ bias,
     int64_t n_tok, int64_t Tlen, int C, const int32_t* __restrict__ cu, int N, int n_l2,
     int group, float l2_eps, const float* __restrict__ cs_in, float* __restrict__ cs_out,
@@ -128,7 +128,7 @@ __global__ void __launch_bounds__(CONV_THREADS) conv_silu_kernel(
         float a = bs[e];
 #pragma unroll
         for (int j = 0; j < K - 1; ++j) a = fmaf(wt[e][j], win[j][e], a);
-        acc[e] = siluf_(fmaf(wt[e][K - 1], xt[e], a));
+        acc[e] = silu_fast(fmaf(wt[e][K - 1], xt[e], a));
       }
 #pragma unroll
       for (int j = 0; j + 1 < K - 1; ++j)

@@ -113,12 +113,13 @@ gdn_status gdn_workspace_status(const void* workspace, void* stream, int* device
   return GDN_OK;
 }
 
-gdn_status gdn_chunk_fwd(const void* q, const void* k, const void* v, const float* g,
-                         const float* beta, gdn_dtype dtype, float scale,
-                         const float* initial_state, const int32_t* cu_seqlens, int N, int B,
-                         int64_t T, int Hk, int Hv, int dk, int dv, int chunk, void* out,
-                         float* final_state, void* workspace, size_t workspace_bytes,
-                         void* stream) {
+gdn_status gdn_chunk_fwd_strided(const void* q, int64_t q_tok_stride, const void* k,
+                                 int64_t k_tok_stride, const void* v, int64_t v_tok_stride,
+                                 const float* g, const float* beta, gdn_dtype dtype, float scale,
+                                 const float* initial_state, const int32_t* cu_seqlens, int N,
+                                 int B, int64_t T, int Hk, int Hv, int dk, int dv, int chunk,
+                                 void* out, float* final_state, void* workspace,
+                                 size_t workspace_bytes, void* stream) {
   if (bad_dtype(dtype) || N < 0 || B < 0 || T < 0 || Hk < 1 || Hv < 1 || dk < 1 || dv < 1)
     return GDN_ERR_INVALID_ARG;
   if (Hv % Hk != 0) return GDN_ERR_INVALID_ARG;
@@ -126,6 +127,11 @@ gdn_status gdn_chunk_fwd(const void* q, const void* k, const void* v, const floa
   if (!(scale == scale)) return GDN_ERR_INVALID_ARG;  // NaN
   if (dk % 16 != 0 || dv % 16 != 0 || dk > 128 || dv > 128) return GDN_ERR_UNSUPPORTED;
   if (chunk != 16 && chunk != 32 && chunk != 64) return GDN_ERR_UNSUPPORTED;
+  // token strides: at least one token's heads, and whole 16-byte rows
+  if (q_tok_stride < (int64_t)Hk * dk || k_tok_stride < (int64_t)Hk * dk ||
+      v_tok_stride < (int64_t)Hv * dv || q_tok_stride % 8 || k_tok_stride % 8 ||
+      v_tok_stride % 8)
+    return GDN_ERR_INVALID_ARG;
   if (!workspace || workspace_bytes < gdn_chunk_fwd_workspace_size(N, B, T, Hk, Hv, dk, dv, chunk))
     return GDN_ERR_INVALID_ARG;
   if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return GDN_ERR_INVALID_ARG;
@@ -146,14 +152,26 @@ gdn_status gdn_chunk_fwd(const void* q, const void* k, const void* v, const floa
   cudaStream_t s = as_stream(stream);
   int* status = reinterpret_cast<int*>(workspace);
   if (cudaMemsetAsync(status, 0, sizeof(int), s) != cudaSuccess) return GDN_ERR_CUDA;
+  const TokStrides ts{q_tok_stride, k_tok_stride, v_tok_stride};
   cudaError_t e;
   if (dtype == GDN_BF16 && dk == 128 && dv == 128 && chunk == 64)
-    e = launch_chunk_tc(q, k, v, g, beta, scale, initial_state, cu_seqlens, N, B, T, Hk, Hv, out,
-                        final_state, status, s);
+    e = launch_chunk_tc(q, k, v, ts, g, beta, scale, initial_state, cu_seqlens, N, B, T, Hk, Hv,
+                        out, final_state, status, s);
   else
-    e = launch_chunk_simt(q, k, v, g, beta, dtype, scale, initial_state, cu_seqlens, N, B, T, Hk,
-                          Hv, dk, dv, chunk, out, final_state, status, s);
+    e = launch_chunk_simt(q, k, v, ts, g, beta, dtype, scale, initial_state, cu_seqlens, N, B, T,
+                          Hk, Hv, dk, dv, chunk, out, final_state, status, s);
   return from_cuda(e);
+}
+
+gdn_status gdn_chunk_fwd(const void* q, const void* k, const void* v, const float* g,
+                         const float* beta, gdn_dtype dtype, float scale,
+                         const float* initial_state, const int32_t* cu_seqlens, int N, int B,
+                         int64_t T, int Hk, int Hv, int dk, int dv, int chunk, void* out,
+                         float* final_state, void* workspace, size_t workspace_bytes,
+                         void* stream) {
+  return gdn_chunk_fwd_strided(q, (int64_t)Hk * dk, k, (int64_t)Hk * dk, v, (int64_t)Hv * dv, g,
+                               beta, dtype, scale, initial_state, cu_seqlens, N, B, T, Hk, Hv, dk,
+                               dv, chunk, out, final_state, workspace, workspace_bytes, stream);
 }
 
 gdn_status gdn_recurrent_step(const void* q, const void* k, const void* v, const float* g,

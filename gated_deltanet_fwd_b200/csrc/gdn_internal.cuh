@@ -103,6 +103,10 @@ __device__ __forceinline__ void load4(const float* p, float (&f)[4]) {
 
 __device__ __forceinline__ float sigmoidf_(float x) { return 1.0f / (1.0f + expf(-x)); }
 __device__ __forceinline__ float siluf_(float x) { return x / (1.0f + expf(-x)); }
+// SiLU for kernels whose result is rounded to bf16: the fast exponential and division intrinsics
+// (relative error ~1e-6, far below bf16's 2^-8) keep these HBM-bound kernels off the ALU roof.
+// For x < -87 the exponential overflows to +inf and the quotient is the correct limit, -0.
+__device__ __forceinline__ float silu_fast(float x) { return __fdividef(x, 1.0f + __expf(-x)); }
 __device__ __forceinline__ float softplusf_(float x) {
   return fmaxf(x, 0.0f) + log1pf(expf(-fabsf(x)));
 }
@@ -145,15 +149,22 @@ cudaError_t launch_recurrent(const void* q, const void* k, const void* v, const 
                              const float* beta, gdn_dtype dt, float scale, float* state, int N,
                              int Hk, int Hv, int dk, int dv, void* out, cudaStream_t s);
 
+// Element distances between consecutive tokens of q, k and v (dense: Hk*dk, Hk*dk, Hv*dv).
+struct TokStrides {
+  int64_t q, k, v;
+};
+
 // CUDA-core chunk path (any supported shape / dtype).
-cudaError_t launch_chunk_simt(const void* q, const void* k, const void* v, const float* g,
+cudaError_t launch_chunk_simt(const void* q, const void* k, const void* v, TokStrides ts,
+                              const float* g,
                               const float* beta, gdn_dtype dt, float scale, const float* S0,
                               const int32_t* cu, int N, int B, int64_t T, int Hk, int Hv, int dk,
                               int dv, int chunk, void* out, float* S_T, int* status,
                               cudaStream_t s);
 
 // Tensor-core chunk path: bf16, dk = dv = 128, chunk = 64.
-cudaError_t launch_chunk_tc(const void* q, const void* k, const void* v, const float* g,
+cudaError_t launch_chunk_tc(const void* q, const void* k, const void* v, TokStrides ts,
+                            const float* g,
                             const float* beta, float scale, const float* S0, const int32_t* cu,
                             int N, int B, int64_t T, int Hk, int Hv, void* out, float* S_T,
                             int* status, cudaStream_t s);

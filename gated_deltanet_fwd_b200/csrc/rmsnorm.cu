@@ -43,7 +43,7 @@ __global__ void __launch_bounds__(256) rmsnorm_gated_kernel(const T* __restrict_
       const float inv = rsqrtf(ss * (1.0f / DIM) + eps);
       float yv[8];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) yv[i] = xv[i] * inv * wv[i] * siluf_(zv[i]);
+      for (int i = 0; i < 8; ++i) yv[i] = xv[i] * inv * wv[i] * silu_fast(zv[i]);
       store8(y + r * DIM + sub * 8, yv);
     }
   }

@@ -32,6 +32,8 @@ SIGNATURES = {
                                     _P, _P]),
     "gdn_chunk_fwd": (_I, [_P, _P, _P, _P, _P, _I, _F, _P, _P, _I, _I, _I64, _I, _I, _I, _I, _I,
                            _P, _P, _P, _SZ, _P]),
+    "gdn_chunk_fwd_strided": (_I, [_P, _I64, _P, _I64, _P, _I64, _P, _P, _I, _F, _P, _P, _I, _I,
+                                   _I64, _I, _I, _I, _I, _I, _P, _P, _P, _SZ, _P]),
     "gdn_chunk_fwd_noalloc": (_I, [_P, _P, _P, _P, _P, _I, _F, _P, _P, _I, _I, _I64, _I, _I, _I,
                                    _I, _I, _P, _P, _P]),
     "gdn_chunk_fwd_workspace_size": (_SZ, [_I, _I, _I64, _I, _I, _I, _I, _I]),
@@ -96,6 +98,16 @@ def _cuda(*ts):
             raise ValueError("tensors must be contiguous CUDA tensors")
 
 
+def _tok_stride(t):
+    """Token stride of a [B, T, H, d] view whose heads are packed inside each token, else None."""
+    B, T, H, d = t.shape
+    if not t.is_cuda or t.stride(3) != 1 or t.stride(2) != d:
+        return None
+    if B > 1 and t.stride(0) != T * t.stride(1):
+        return None
+    return t.stride(1)
+
+
 # ------------------------------------------------------------------------------ calls ------
 
 def gdn_gates(a, b, A_log, dt_bias, g=None, beta=None):
@@ -144,23 +156,34 @@ def gdn_chunk_fwd(q, k, v, g, beta, scale=None, initial_state=None, cu_seqlens=N
     """Chunked prefill: (q, k, v, g, beta, initial_state, cu_seqlens) -> (out, final_state).
 
     q, k: [B, T, Hk, dk]; v: [B, T, Hv, dv]; g, beta: [B, T, Hv] fp32; states [N, Hv, dv, dk].
+    q, k, v may be views whose tokens are not packed back to back (e.g. slices of the conv's
+    [q | k | v] output); those go through gdn_chunk_fwd_strided.
     """
-    _cuda(q, k, v, g, beta, initial_state, cu_seqlens, out, final_state, workspace)
+    _cuda(g, beta, initial_state, cu_seqlens, out, final_state, workspace)
+    qs, ks, vs = _tok_stride(q), _tok_stride(k), _tok_stride(v)
+    if qs is None or ks is None or vs is None:
+        raise ValueError("q, k, v must be CUDA [B, T, H, d] tensors with each token's heads packed")
     B, T, Hk, dk = q.shape
     Hv, dv = v.shape[2], v.shape[3]
     N = cu_seqlens.numel() - 1 if cu_seqlens is not None else B
     scale = dk ** -0.5 if scale is None else scale
-    out = torch.empty_like(v) if out is None else out
+    out = torch.empty(v.shape, dtype=v.dtype, device=v.device) if out is None else out
     if final_state is None and output_final_state:
         final_state = torch.empty((N, Hv, dv, dk), dtype=torch.float32, device=q.device)
     ws_bytes = workspace_size(N, B, T, Hk, Hv, dk, dv, chunk)
     if workspace is None:
         workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=q.device)
-    _check("gdn_chunk_fwd", load().gdn_chunk_fwd(
-        _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _dt(q), float(scale),
-        _ptr(initial_state), _ptr(cu_seqlens), N, B, T, Hk, Hv, dk, dv, chunk, _ptr(out),
-        _ptr(final_state), _ptr(workspace), workspace.numel() * workspace.element_size(),
-        _stream(q)))
+    ws_b = workspace.numel() * workspace.element_size()
+    if (qs, ks, vs) == (Hk * dk, Hk * dk, Hv * dv):
+        _check("gdn_chunk_fwd", load().gdn_chunk_fwd(
+            _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _dt(q), float(scale),
+            _ptr(initial_state), _ptr(cu_seqlens), N, B, T, Hk, Hv, dk, dv, chunk, _ptr(out),
+            _ptr(final_state), _ptr(workspace), ws_b, _stream(q)))
+    else:
+        _check("gdn_chunk_fwd_strided", load().gdn_chunk_fwd_strided(
+            _ptr(q), qs, _ptr(k), ks, _ptr(v), vs, _ptr(g), _ptr(beta), _dt(q), float(scale),
+            _ptr(initial_state), _ptr(cu_seqlens), N, B, T, Hk, Hv, dk, dv, chunk, _ptr(out),
+            _ptr(final_state), _ptr(workspace), ws_b, _stream(q)))
     return out, final_state
 
 

@@ -127,6 +127,24 @@ gdn_status gdn_chunk_fwd(const void* q, const void* k, const void* v, const floa
                          void* stream);
 
 /*
+ * gdn_chunk_fwd_strided -- gdn_chunk_fwd on q, k, v whose tokens are not packed back to back,
+ * e.g. q, k and v read straight out of the [q | k | v] output of gdn_causal_conv1d_silu (the
+ * split after the conv in [P3]'s flowchart) without copying them apart.
+ * q_tok_stride, k_tok_stride, v_tok_stride: elements between consecutive tokens (batch row b,
+ * token t sits at token index b*T + t); within a token the heads stay contiguous (head h at
+ * h*dk, resp. h*dv).  Each stride must be >= the token's heads (Hk*dk, resp. Hv*dv) and a
+ * multiple of 8 elements.  Everything else as gdn_chunk_fwd, which is this call with the dense
+ * strides Hk*dk, Hk*dk, Hv*dv.  out stays dense [B, T, Hv, dv].
+ */
+gdn_status gdn_chunk_fwd_strided(const void* q, int64_t q_tok_stride, const void* k,
+                                 int64_t k_tok_stride, const void* v, int64_t v_tok_stride,
+                                 const float* g, const float* beta, gdn_dtype dtype, float scale,
+                                 const float* initial_state, const int32_t* cu_seqlens, int N,
+                                 int B, int64_t T, int Hk, int Hv, int dk, int dv, int chunk,
+                                 void* out, float* final_state, void* workspace,
+                                 size_t workspace_bytes, void* stream);
+
+/*
  * gdn_chunk_fwd_noalloc -- gdn_chunk_fwd for callers that cannot allocate device memory.  The
  * pages have no counterpart: this is a library convenience.
  * Who needs it: code that receives device pointers from another runtime and may not allocate

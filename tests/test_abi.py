@@ -113,6 +113,21 @@ def test_chunk_rejections(lib):
 
 
 @fake_ptr_only_without_gpu
+def test_chunk_strided_rejections(lib):
+    f = lib.gdn_chunk_fwd_strided
+
+    def call(qs=2048, ks=2048, vs=4096, Hk=16, Hv=32, dk=128, dv=128):
+        return f(A16, qs, A16, ks, A16, vs, A16, A16, 0, 0.1, NUL, NUL, 1, 1, 64, Hk, Hv, dk, dv,
+                 64, A16, A16, A16, 256, STREAM)
+
+    E = gdn.GDN_ERR_INVALID_ARG
+    assert call(qs=2040) == E       # smaller than one token's heads
+    assert call(ks=2052) == E       # not a multiple of 8 elements
+    assert call(vs=4092) == E
+    assert call(vs=0) == E
+
+
+@fake_ptr_only_without_gpu
 def test_recurrent_rejections(lib):
     f = lib.gdn_recurrent_step
 

@@ -135,3 +135,24 @@ def test_prefill_varlen_32k_sampled():
 
 def test_prefill_varlen_32k_slow_decay_sampled():
     _sampled("prefill_varlen_32k", [(0, 5), (3, 16)], a_mean=-6.0)
+
+
+@pytest.mark.parametrize("chunk,dtype", [(64, "bf16"), (32, "bf16"), (16, "f32")])
+def test_chunk_on_conv_output_views(chunk, dtype):
+    """q, k, v as strided views into one [B, T, Hk*dk | Hk*dk | Hv*dv] buffer (the conv's output
+    layout), read in place through gdn_chunk_fwd_strided; must equal the dense call exactly."""
+    B, T, Hk, Hv, d = 2, 150, 2, 4, 128
+    x = inputs.rule_inputs(B=B, T=T, Hk=Hk, Hv=Hv, dk=d, dv=d, dtype=dtype, seed=31,
+                           s0_std=0.02, a_mean=-6.0)
+    g, beta = oracle_gates_f32(x)
+    mix = torch.cat([x["q"].reshape(B, T, -1), x["k"].reshape(B, T, -1),
+                     x["v"].reshape(B, T, -1)], dim=-1).to(DEV)
+    qv = mix[:, :, :Hk * d].view(B, T, Hk, d)
+    kv = mix[:, :, Hk * d:2 * Hk * d].view(B, T, Hk, d)
+    vv = mix[:, :, 2 * Hk * d:].view(B, T, Hv, d)
+    S0 = x["initial_state"].to(DEV)
+    o1, S1 = gdn.gdn_chunk_fwd(qv, kv, vv, g.to(DEV), beta.to(DEV), initial_state=S0,
+                               chunk=chunk)
+    o2, S2 = gdn.gdn_chunk_fwd(x["q"].to(DEV), x["k"].to(DEV), x["v"].to(DEV), g.to(DEV),
+                               beta.to(DEV), initial_state=S0, chunk=chunk)
+    assert torch.equal(o1, o2) and torch.equal(S1, S2)
