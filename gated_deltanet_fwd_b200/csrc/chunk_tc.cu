@@ -70,7 +70,8 @@ constexpr uint32_t PR_TPL = 139264;                   // 2 x [T'; P] staging til
 // mbarriers (same offsets in both CTAs; each CTA initialises and uses its own subset)
 constexpr uint32_t OFF_BAR = 180224;
 constexpr uint32_t N_BARS = 16;
-constexpr uint32_t SMEM_USED = OFF_BAR + N_BARS * 8 + 16;
+constexpr uint32_t OFF_GX = OFF_BAR + 256;  // prefetched gates: 2 x (g[64], beta[64]) fp32
+constexpr uint32_t SMEM_USED = OFF_GX + 1024;
 constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;  // slack for 1024-byte alignment
 static_assert(PR_PV + 512 <= PR_TPL && PR_TPL % 1024 == 0, "prep layout");
 static_assert(PR_TPL + 2 * TP_BUF <= OFF_BAR, "prep staging");
@@ -166,6 +167,16 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
+// Descriptor of the same operand tile `bytes` further on (start-address field, 16-byte units;
+// shared-memory addresses stay below 256 KB, so the field never carries).
+__device__ __forceinline__ uint64_t dadd(uint64_t d, uint32_t bytes) {
+  return d + (uint64_t)(bytes >> 4);
+}
+// K-major 128-byte-swizzled operand with two 64-element K halves `half` bytes apart: k-step ks.
+__device__ __forceinline__ uint32_t kstep_kmajor(int ks, uint32_t half) {
+  return (uint32_t)(ks >> 2) * half + (uint32_t)(ks & 3) * 32u;
+}
+
 // ---------------------------------------------------------------- cluster helpers ----------
 
 __device__ __forceinline__ uint32_t cluster_rank() {
@@ -186,41 +197,23 @@ __device__ __forceinline__ uint32_t peer_addr(uint32_t local, uint32_t rank) {
   return r;
 }
 
-// Arrive on an mbarrier of a peer CTA, releasing this thread's prior writes at cluster scope.
+// Arrive on an mbarrier of a peer CTA (release at CTA scope: used only to hand back a buffer
+// whose readers, this CTA's MMAs, have completed).
 __device__ __forceinline__ void mbar_arrive_peer(uint32_t peer_bar) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(peer_bar)
-               : "memory");
+  asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(peer_bar) : "memory");
 }
 
-// Bounded wait on a local mbarrier that a peer CTA arrives on (acquire at cluster scope).
-__device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity) {
-  const uint32_t a = smem_u32(bar);
-  auto poll = [&]() {
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2, %3;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(a), "r"(parity), "r"(1000000u)
-        : "memory");
-    return ok != 0;
-  };
-  if (poll()) return true;
-  const uint64_t t0 = globaltimer_ns();
-  for (uint32_t i = 0; i < kSpinLimit; ++i) {
-    if (poll()) return true;
-    if ((i & 63) == 63 && globaltimer_ns() - t0 > kWaitLimitNs) return false;
-  }
-  return false;
-}
-
-// Arms a peer CTA's mbarrier with one arrival plus `bytes` of expected transaction count.
-__device__ __forceinline__ void mbar_arrive_expect_tx_peer(uint32_t peer_bar, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.release.cluster.shared::cluster.b64 _, [%0], %1;" ::"r"(
-                   peer_bar),
-               "r"(bytes)
+// 4-byte asynchronous global -> shared copy; `valid` false writes zero instead.
+__device__ __forceinline__ void cp_async4(uint32_t dst, const float* src, bool valid) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(dst), "l"(src),
+               "r"(valid ? 4 : 0)
                : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.wait_all;" ::: "memory");
 }
 
 // Copies `bytes` of this CTA's shared memory into a peer CTA's shared memory; the bytes are
@@ -283,6 +276,11 @@ __global__ void __launch_bounds__(TC_THREADS, 1) chunk_tc_kernel(
     mbar_init(&bars[B_DRAIN], 1);
     *abort_flag = 0;
     fence_barrier_init();
+    // the chain CTA expects one [T'; P] tile per chunk from the prep CTA's bulk copies
+    if (rank == 1) {
+      for (int i = 0; i < 2 && i < nchunks; ++i)
+        mbar_arrive_expect_tx(&bars[B_PREP_FULL0 + i], TP_BUF);
+    }
   }
   if (warp == 0) {
     tmem_alloc(tmem_slot, rank == 1 ? 512 : 64);
@@ -344,15 +342,23 @@ __global__ void __launch_bounds__(TC_THREADS, 1) chunk_tc_kernel(
     float* gl2 = reinterpret_cast<float*>(smem + PR_PV);  // gamma * log2(e) of the chunk
     float* bet = gl2 + 64;
     const uint32_t id_d1 = idesc_bf16(128, 64, 0, 0);
-    // gates of the next chunk are fetched one chunk ahead (warp 0, rows lane and 32 + lane)
-    float pf_g0 = 0.0f, pf_g1 = 0.0f, pf_b0 = 0.0f, pf_b1 = 0.0f;
+    const uint64_t dkq0 = sdesc_sw128(sbase + PR_KQ, 16, 1024);
+    // gates of the next chunk are fetched one chunk ahead by warp 0 (asynchronous copies into
+    // gx[c & 1]: g of rows 0..63, then beta); rows past the sequence end read as zero
+    const float* gx = reinterpret_cast<const float*>(smem + OFF_GX);
     auto fetch_gates = [&](int c) {
       const int64_t tc = s_beg + 64 * c;
       const int Lc = (int)min((int64_t)64, s_end - tc);
-      pf_g0 = lane < Lc ? __ldg(P.g + (tc + lane) * P.Hv + h) : 0.0f;
-      pf_g1 = 32 + lane < Lc ? __ldg(P.g + (tc + 32 + lane) * P.Hv + h) : 0.0f;
-      pf_b0 = lane < Lc ? __ldg(P.beta + (tc + lane) * P.Hv + h) : 0.0f;
-      pf_b1 = 32 + lane < Lc ? __ldg(P.beta + (tc + 32 + lane) * P.Hv + h) : 0.0f;
+      const uint32_t dst = sbase + OFF_GX + (uint32_t)(c & 1) * 512u;
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        const int rr = 32 * hh + lane;
+        const bool v = rr < Lc;
+        const int64_t off = v ? (tc + rr) * P.Hv + h : 0;
+        cp_async4(dst + 4u * rr, P.g + off, v);
+        cp_async4(dst + 256u + 4u * rr, P.beta + off, v);
+      }
+      cp_async_commit();
     };
     if (warp == 0 && nchunks > 0) fetch_gates(0);
     TC_TRACE_DECL(leader);
@@ -367,11 +373,11 @@ __global__ void __launch_bounds__(TC_THREADS, 1) chunk_tc_kernel(
         TC_TS(8);
         if (ok) {
           tc_fence_after();
-          const uint32_t kqa = sbase + PR_KQ + st * KQ_STAGE;
+          const uint64_t dkq = dadd(dkq0, st * KQ_STAGE);
+#pragma unroll
           for (int ks = 0; ks < 8; ++ks) {
-            const uint32_t half = kqa + (uint32_t)(ks >> 2) * 16384u + (uint32_t)(ks & 3) * 32u;
-            mma_bf16_ss(tmem, sdesc_sw128(half, 16, 1024), sdesc_sw128(half, 16, 1024), id_d1,
-                        ks > 0);
+            const uint64_t d = dadd(dkq, kstep_kmajor(ks, 16384));
+            mma_bf16_ss(tmem, d, d, id_d1, ks > 0);
           }
           mma_commit(&bars[B_D1_FULL]);
         }
@@ -380,7 +386,11 @@ __global__ void __launch_bounds__(TC_THREADS, 1) chunk_tc_kernel(
       // cumulative log-decays and write strengths while D1 runs; rows past the sequence end carry
       // zero log-decay and zero beta, which makes their corrections exactly zero
       if (warp == 0) {
-        float x0 = pf_g0, x1 = pf_g1;
+        cp_async_wait_all();
+        __syncwarp();
+        const float* gc = gx + (c & 1) * 128;
+        float x0 = gc[lane], x1 = gc[32 + lane];
+        const float b0 = gc[64 + lane], b1 = gc[96 + lane];
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
           const float y0 = __shfl_up_sync(0xffffffffu, x0, o);
@@ -393,14 +403,15 @@ __global__ void __launch_bounds__(TC_THREADS, 1) chunk_tc_kernel(
         x1 += __shfl_sync(0xffffffffu, x0, 31);
         gl2[lane] = x0 * kLog2e;
         gl2[32 + lane] = x1 * kLog2e;
-        bet[lane] = pf_b0;
-        bet[32 + lane] = pf_b1;
+        bet[lane] = b0;
+        bet[32 + lane] = b1;
+        __syncwarp();
         if (c + 1 < nchunks) fetch_gates(c + 1);
       }
       TC_TS(0);
       // the chain CTA has released this chunk's [T'; P] buffer (the leader waits; the barrier
       // below orders everyone's writes after it)
-      if (leader) ok = ok && mbar_wait_cluster(&bars[B_PREP_EMPTY0 + b], ((c >> 1) & 1) ^ 1);
+      if (leader) ok = ok && mbar_wait(&bars[B_PREP_EMPTY0 + b], ((c >> 1) & 1) ^ 1);
       ok = ok && mbar_wait(&bars[B_D1_FULL], c & 1);
       if (leader && ok) mbar_arrive(&bars[B_EMPTY0 + st]);  // D1 has read this stage
       // one decision for all prep threads; also makes gl2 / bet visible to them
@@ -455,13 +466,19 @@ __global__ void __launch_bounds__(TC_THREADS, 1) chunk_tc_kernel(
       if (warp < 2) {
         const int blk = 2 * warp + (lane >> 4), jj = lane & 15, col = 16 * blk + jj;
         const float* ab = Af + 16 * blk * AS + 16 * blk;
-        float x[16];
+        float x[16], a[16], an[16];
 #pragma unroll
         for (int r = 0; r < 16; ++r) x[r] = (r == jj) ? 1.0f : 0.0f;
 #pragma unroll
+        for (int t = 1; t < 16; ++t) a[t] = ab[t * AS];
+#pragma unroll
         for (int r = 0; r < 15; ++r) {
 #pragma unroll
-          for (int t = r + 1; t < 16; ++t) x[t] = fmaf(-ab[t * AS + r], x[r], x[t]);
+          for (int t = r + 2; t < 16; ++t) an[t] = ab[t * AS + r + 1];  // next column, early
+#pragma unroll
+          for (int t = r + 1; t < 16; ++t) x[t] = fmaf(-a[t], x[r], x[t]);
+#pragma unroll
+          for (int t = r + 2; t < 16; ++t) a[t] = an[t];
         }
 #pragma unroll
         for (int r = 0; r < 16; ++r) Tf[(16 * blk + r) * AS + col] = x[r];
@@ -544,15 +561,14 @@ __global__ void __launch_bounds__(TC_THREADS, 1) chunk_tc_kernel(
       TC_TS(11);
       named_bar(1, TC_WORKERS);
       TC_TS(12);
-      if (leader) {
-        const uint32_t full_peer = peer_addr(smem_u32(&bars[B_PREP_FULL0 + b]), 1);
-        mbar_arrive_expect_tx_peer(full_peer, TP_BUF);
+      // the chain CTA arms its barrier for these bytes itself; the copy only completes them
+      if (leader)
         bulk_copy_to_peer(peer_addr(sbase + CH_TP + b * TP_BUF, 1), smem_u32(tpl), TP_BUF,
-                          full_peer);
-      }
+                          peer_addr(smem_u32(&bars[B_PREP_FULL0 + b]), 1));
       TC_TS(6);
     }
     TC_TRACE_FLUSH(2);
+    if (warp == 0) cp_async_wait_all();  // no gate copy may still be landing at exit
     if (leader) {
       mma_commit(&bars[B_DRAIN]);
       mbar_wait(&bars[B_DRAIN], 0);
@@ -568,6 +584,13 @@ __global__ void __launch_bounds__(TC_THREADS, 1) chunk_tc_kernel(
     const uint32_t id_ks = idesc_bf16(128, 128, 0, 1);
     const uint32_t id_u = idesc_bf16(128, 128, 0, 1);
     const uint32_t id_s = idesc_bf16(128, 128, 1, 1);
+    // operand descriptors at each tile's first k-step
+    const uint64_t dKQ = sdesc_sw128(sbase + CH_KQ, 16, 1024);       // [K; Q] (K-major)
+    const uint64_t dKT = sdesc_sw128(sbase + CH_KQ, 16384, 1024);    // K^T (MN-major)
+    const uint64_t dSB = sdesc_sw128(sbase + CH_SB, 16384, 1024);    // S^T (MN-major)
+    const uint64_t dTP = sdesc_sw128(sbase + CH_TP, 16, 1024);       // [T'; P] (K-major)
+    const uint64_t dXU = sdesc_sw128(sbase + CH_XU, 8192, 1024);     // X, then U (MN-major)
+    const uint64_t dDU = sdesc_sw128(sbase + CH_V, 8192, 1024);      // D U (MN-major)
     // The fp32 state lives in tensor memory (TM_S: lane i = row of S^T, 128 value columns); this
     // thread owns lane i, columns jb..jb+31.  Its bf16 copy in shared memory is step 1's operand.
     const size_t sbase_g = ((size_t)n * P.Hv + h) * 128 * 128;
@@ -583,19 +606,29 @@ __global__ void __launch_bounds__(TC_THREADS, 1) chunk_tc_kernel(
       *reinterpret_cast<uint4*>(sb + sw128(i, jo + 16 * pc)) = pack8(&v16[0]);
       *reinterpret_cast<uint4*>(sb + sw128(i, jo + 16 * pc + 8)) = pack8(&v16[8]);
     }
+    // log-decays of the next chunk are fetched one chunk ahead by warp 0 (asynchronous copies
+    // into gx[c & 1], complete before the chunk's last barrier); rows past the end read as zero
+    const float* gx = reinterpret_cast<const float*>(smem + OFF_GX);
+    auto fetch_g = [&](int c) {
+      const int64_t tc = s_beg + 64 * c;
+      const int Lc = (int)min((int64_t)64, s_end - tc);
+      const uint32_t dst = sbase + OFF_GX + (uint32_t)(c & 1) * 256u;
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        const int rr = 32 * hh + lane;
+        const bool v = rr < Lc;
+        cp_async4(dst + 4u * rr, P.g + (v ? (tc + rr) * P.Hv + h : 0), v);
+      }
+      cp_async_commit();
+    };
+    if (warp == 0 && nchunks > 0) {
+      fetch_g(0);
+      cp_async_wait_all();
+    }
     tmem_st_wait();
     fence_proxy_async_smem();
     tc_fence_before();
     named_bar(1, TC_WORKERS);
-    // log-decays of the next chunk are fetched one chunk ahead (rows lane and 32 + lane)
-    float pg0 = 0.0f, pg1 = 0.0f;
-    auto fetch_g = [&](int c) {
-      const int64_t tc = s_beg + 64 * c;
-      const int Lc = (int)min((int64_t)64, s_end - tc);
-      pg0 = lane < Lc ? __ldg(P.g + (tc + lane) * P.Hv + h) : 0.0f;
-      pg1 = 32 + lane < Lc ? __ldg(P.g + (tc + 32 + lane) * P.Hv + h) : 0.0f;
-    };
-    if (nchunks > 0) fetch_g(0);
     TC_TRACE_DECL(leader || e == 64);
 
     // Exits are decided jointly (named_bar_and): a wait that ran out in any thread makes all 512
@@ -605,12 +638,10 @@ __global__ void __launch_bounds__(TC_THREADS, 1) chunk_tc_kernel(
       const uint32_t par = c & 1;
       const int64_t t0 = s_beg + 64 * c;
       const int L = (int)min((int64_t)64, s_end - t0);
-      const uint32_t kqa = sbase + CH_KQ + st * KQ_STAGE;
-      const uint32_t tpa = sbase + CH_TP + b * TP_BUF;
       unsigned char* vt = smem + CH_V + st * V_STAGE;
       TC_TS(7);
       // in-chunk cumulative log-decay (inclusive scan over the chunk's 64 rows)
-      float gl = pg0, gh = pg1;
+      float gl = gx[(c & 1) * 64 + lane], gh = gx[(c & 1) * 64 + 32 + lane];
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
         const float y0 = __shfl_up_sync(0xffffffffu, gl, o);
@@ -622,7 +653,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) chunk_tc_kernel(
       }
       gh += __shfl_sync(0xffffffffu, gl, 31);
       const float glast = __shfl_sync(0xffffffffu, gh, 31);
-      if (c + 1 < nchunks) fetch_g(c + 1);
+      if (warp == 0 && c + 1 < nchunks) fetch_g(c + 1);
       // this thread's row r: i for rows 0..63, i - 64 for rows 64..127
       const float g_row = __expf((ew & 1) ? gh : gl);           // Gamma_r
       const float d_row = __expf(glast - ((ew & 1) ? gh : gl)); // e^{gamma_63 - gamma_r}
@@ -633,12 +664,11 @@ __global__ void __launch_bounds__(TC_THREADS, 1) chunk_tc_kernel(
       // step 1: D_KS = [K; Q] S0^T
       if (leader && ok) {
         tc_fence_after();
-        for (int ks = 0; ks < 8; ++ks) {
-          const uint32_t a = kqa + (uint32_t)(ks >> 2) * 16384u + (uint32_t)(ks & 3) * 32u;
-          const uint32_t bb = sbase + CH_SB + (uint32_t)ks * 2048u;
-          mma_bf16_ss(tmem + TM_KS, sdesc_sw128(a, 16, 1024), sdesc_sw128(bb, 16384, 1024), id_ks,
+        const uint64_t da = dadd(dKQ, st * KQ_STAGE);
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks)
+          mma_bf16_ss(tmem + TM_KS, dadd(da, kstep_kmajor(ks, 16384)), dadd(dSB, ks * 2048), id_ks,
                       ks > 0);
-        }
         mma_commit(&bars[B_M_KS]);
       }
       // S <- Gamma_L S in tensor memory while step 1 runs (step 5 then accumulates onto it; the
@@ -685,15 +715,16 @@ __global__ void __launch_bounds__(TC_THREADS, 1) chunk_tc_kernel(
       }
       TC_TS(2);
       // step 3: D_U = [T'; P] X  (needs this chunk's T' and P from the prep CTA)
-      ok = !leader || mbar_wait_cluster(&bars[B_PREP_FULL0 + b], (c >> 1) & 1);
+      ok = !leader || mbar_wait(&bars[B_PREP_FULL0 + b], (c >> 1) & 1);
+      // re-arm the buffer's barrier for chunk c + 2, whose copy the prep CTA can only start
+      // after this chunk hands the buffer back
+      if (leader && ok && c + 2 < nchunks) mbar_arrive_expect_tx(&bars[B_PREP_FULL0 + b], TP_BUF);
       if (leader && ok) {
         tc_fence_after();
-        for (int ks = 0; ks < 4; ++ks) {
-          const uint32_t a = tpa + (uint32_t)ks * 32u;
-          const uint32_t bb = sbase + CH_XU + (uint32_t)ks * 2048u;
-          mma_bf16_ss(tmem + TM_U, sdesc_sw128(a, 16, 1024), sdesc_sw128(bb, 8192, 1024), id_u,
-                      ks > 0);
-        }
+        const uint64_t dt = dadd(dTP, b * TP_BUF);
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks)
+          mma_bf16_ss(tmem + TM_U, dadd(dt, ks * 32), dadd(dXU, ks * 2048), id_u, ks > 0);
         mma_commit(&bars[B_M_U]);
       }
       ok = ok && mbar_wait(&bars[B_M_U], par);
@@ -728,18 +759,15 @@ __global__ void __launch_bounds__(TC_THREADS, 1) chunk_tc_kernel(
       // steps 3b and 5: D_U = [T'; P] U (rows 64..127 are P U);  D_S += K^T (D U)
       if (leader) {
         tc_fence_after();
-        for (int ks = 0; ks < 4; ++ks) {
-          const uint32_t a = tpa + (uint32_t)ks * 32u;
-          const uint32_t bb = sbase + CH_XU + (uint32_t)ks * 2048u;
-          mma_bf16_ss(tmem + TM_U, sdesc_sw128(a, 16, 1024), sdesc_sw128(bb, 8192, 1024), id_u,
-                      ks > 0);
-        }
-        for (int ks = 0; ks < 4; ++ks) {
-          const uint32_t a = kqa + (uint32_t)ks * 2048u;
-          const uint32_t bb = sbase + CH_V + st * V_STAGE + (uint32_t)ks * 2048u;
-          mma_bf16_ss(tmem + TM_S, sdesc_sw128(a, 16384, 1024), sdesc_sw128(bb, 8192, 1024), id_s,
-                      1);
-        }
+        const uint64_t dt = dadd(dTP, b * TP_BUF);
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks)
+          mma_bf16_ss(tmem + TM_U, dadd(dt, ks * 32), dadd(dXU, ks * 2048), id_u, ks > 0);
+        const uint64_t dk = dadd(dKT, st * KQ_STAGE);
+        const uint64_t dd = dadd(dDU, st * V_STAGE);
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks)
+          mma_bf16_ss(tmem + TM_S, dadd(dk, ks * 2048), dadd(dd, ks * 2048), id_s, 1);
         mma_commit(&bars[B_M_S]);
         mma_commit(&bars[B_EMPTY0 + st]);
       }
@@ -780,6 +808,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) chunk_tc_kernel(
         fence_proxy_async_smem();
         TC_TS(11);
       }
+      if (warp == 0) cp_async_wait_all();  // next chunk's log-decays, visible after the barrier
       tc_fence_before();
       if (!named_bar_and(1, TC_WORKERS, ok)) {
         fail(GDN_ERR_TIMEOUT);
@@ -788,6 +817,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) chunk_tc_kernel(
       TC_TS(6);
     }
     TC_TRACE_FLUSH(leader ? 3 : 4);
+    if (warp == 0) cp_async_wait_all();  // no gate copy may still be landing at exit
     if (leader) {
       mma_commit(&bars[B_DRAIN]);
       mbar_wait(&bars[B_DRAIN], 0);
