@@ -19,6 +19,7 @@ whole-job value = units of all ranks / max-over-ranks time.
 from __future__ import annotations
 
 import argparse
+import hashlib
 import json
 import math
 import os
@@ -40,6 +41,34 @@ METRIC = "gated-delta-rule prefill tokens/s (T=32K) & decode seqs/s; % of roofli
 # 8*C*d (K K^T, Q K^T, the triangular apply, the intra-chunk output) + 6*d^2 (K S^T, Q S^T and the
 # state update) multiply-adds x 2 = 163,840 FLOP.
 CHUNK_FLOP_PER_TOKEN_HEAD = 8 * 64 * 128 + 6 * 128 * 128
+
+
+# DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of the dominant kernels, from one ncu
+# capture each (summaries under profiles/), tied to the kernel source they were taken from: once
+# the source changes the bench reports traffic as null until it is captured again.
+MEASURED_TRAFFIC = {
+    # chunk_tc_kernel on B=1, T=4096 (prefill 4K): 68.2 MB read + 7.4 MB written = 18,455 B per
+    # token over all 32 heads; scaled by the tokens of a launch (reads scale with tokens; the
+    # write count is a lower bound, the output drains from L2 after the kernel).
+    "gdn_chunk_fwd": dict(source="csrc/chunk_tc.cu", sha256_16="9357e5e1e408224c",
+                          bytes_per_token=75590144 / 4096),
+    # recurrent_step_kernel on 256 sequences x 32 heads: 5.92 TB/s x 172.8 us.
+    "gdn_recurrent_step": dict(source="csrc/recurrent.cu", sha256_16="b07ec22be73c2392",
+                               bytes_per_launch=1.0224e9),
+}
+
+
+def _traffic(kernel, units):
+    m = MEASURED_TRAFFIC[kernel]
+    path = os.path.join(ROOT, "gated_deltanet_fwd_b200", m["source"])
+    try:
+        with open(path, "rb") as f:
+            sha = hashlib.sha256(f.read()).hexdigest()[:16]
+    except OSError:
+        return None
+    if sha != m["sha256_16"]:
+        return None
+    return m.get("bytes_per_launch", m.get("bytes_per_token", 0.0) * units)
 
 
 def _peaks():
@@ -231,7 +260,8 @@ def bench_prefill(dist, gdn, K, W, peaks):
     res = dict(value=tokens * K / (ms * 1e-3), ms_per_step=ms / K, chunk_ms=chunk_ms,
                roofline=dict(bound="tensor", kernel="gdn_chunk_fwd", achieved=achieved,
                              peak=peaks["bf16"], unit="TFLOP/s", frac=achieved / peaks["bf16"],
-                             traffic=None, flop_per_launch=flop,
+                             traffic=_traffic("gdn_chunk_fwd", T),
+                             traffic_unit="bytes per launch", flop_per_launch=flop,
                              peak_source=peaks["source"] + " bf16 burst"),
                gpu_launches=2 * K)
 
@@ -295,7 +325,9 @@ def bench_decode(dist, gdn, K, W, peaks):
                 ms_per_step=ms / K, decode_token_us=rec_ms * 1e3,
                 roofline=dict(bound="hbm", kernel="gdn_recurrent_step", achieved=achieved,
                               peak=peaks["hbm"], unit="GB/s", frac=achieved / peaks["hbm"],
-                              frac_of_nominal_8tbs=achieved / 8000.0, traffic=None,
+                              frac_of_nominal_8tbs=achieved / 8000.0,
+                              traffic=_traffic("gdn_recurrent_step", 0),
+                              traffic_unit="bytes per launch",
                               bytes_per_launch=bytes_per_launch,
                               peak_source=peaks["source"] + " HBM copy"),
                 gpu_launches=2 * steps * K)
