@@ -93,7 +93,9 @@ enum {
 static_assert(B_COUNT <= (int)N_BARS, "barrier space");
 
 // tensor-memory columns (chain CTA; the prep CTA holds D1 only)
-constexpr uint32_t TM_KS = 0, TM_U = 128, TM_S = 256;
+// D_KS alternates between two column blocks by chunk parity, so that a chunk's output can be read
+// out while the next chunk's first MMA runs.
+constexpr uint32_t TM_KS = 0, TM_U = 128, TM_S = 256, TM_KS2 = 384;
 
 constexpr float kLog2e = 1.4426950408889634f;
 
@@ -631,11 +633,39 @@ __global__ void __launch_bounds__(TC_THREADS, 1) chunk_tc_kernel(
     named_bar(1, TC_WORKERS);
     TC_TRACE_DECL(leader || e == 64);
 
+    // O = scale (Gamma_r (Q S0^T)_r + (P U)_r) of chunk c, rows r = i - 64 (threads of rows
+    // 64..127), columns jb..jb+31
+    auto write_out = [&](int c, float g_r) {
+      const int64_t t0 = s_beg + 64 * c;
+      const int L = (int)min((int64_t)64, s_end - t0);
+      const int r = i - 64;
+      const uint32_t tk = (c & 1) ? TM_KS2 : TM_KS;
+      float qs[32], pu[32];
+      tmem_ld16(tmem + tk + jb + lane_off, *reinterpret_cast<float(*)[16]>(qs));
+      tmem_ld16(tmem + tk + jb + 16 + lane_off, *reinterpret_cast<float(*)[16]>(qs + 16));
+      tmem_ld16(tmem + TM_U + jb + lane_off, *reinterpret_cast<float(*)[16]>(pu));
+      tmem_ld16(tmem + TM_U + jb + 16 + lane_off, *reinterpret_cast<float(*)[16]>(pu + 16));
+      tmem_ld_wait();
+      if (r < L) {
+        __nv_bfloat16* orow = P.out + ((t0 + r) * P.Hv + h) * 128 + jb;
+#pragma unroll
+        for (int c8 = 0; c8 < 4; ++c8) {
+          float f[8];
+#pragma unroll
+          for (int q = 0; q < 8; ++q) f[q] = P.scale * fmaf(g_r, qs[8 * c8 + q], pu[8 * c8 + q]);
+          *reinterpret_cast<uint4*>(orow + 8 * c8) = pack8(f);
+        }
+      }
+    };
+    float g_row_prev = 0.0f;
+    bool all_ok = true;
+
     // Exits are decided jointly (named_bar_and): a wait that ran out in any thread makes all 512
     // leave at the same barrier.
     for (int c = 0; c < nchunks; ++c) {
       const int st = c & 1, b = c & 1;
       const uint32_t par = c & 1;
+      const uint32_t tm_ks = (c & 1) ? TM_KS2 : TM_KS;
       const int64_t t0 = s_beg + 64 * c;
       const int L = (int)min((int64_t)64, s_end - t0);
       unsigned char* vt = smem + CH_V + st * V_STAGE;
@@ -667,7 +697,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) chunk_tc_kernel(
         const uint64_t da = dadd(dKQ, st * KQ_STAGE);
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks)
-          mma_bf16_ss(tmem + TM_KS, dadd(da, kstep_kmajor(ks, 16384)), dadd(dSB, ks * 2048), id_ks,
+          mma_bf16_ss(tmem + tm_ks, dadd(da, kstep_kmajor(ks, 16384)), dadd(dSB, ks * 2048), id_ks,
                       ks > 0);
         mma_commit(&bars[B_M_KS]);
       }
@@ -689,8 +719,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1) chunk_tc_kernel(
         // X = V - Gamma_r (K S0^T), rows r = i, columns jb..jb+31
         float ks[32];
         uint4 vraw[4];
-        tmem_ld16(tmem + TM_KS + jb + lane_off, *reinterpret_cast<float(*)[16]>(ks));
-        tmem_ld16(tmem + TM_KS + jb + 16 + lane_off, *reinterpret_cast<float(*)[16]>(ks + 16));
+        tmem_ld16(tmem + tm_ks + jb + lane_off, *reinterpret_cast<float(*)[16]>(ks));
+        tmem_ld16(tmem + tm_ks + jb + 16 + lane_off, *reinterpret_cast<float(*)[16]>(ks + 16));
 #pragma unroll
         for (int c8 = 0; c8 < 4; ++c8)
           vraw[c8] = *reinterpret_cast<const uint4*>(vt + jh * 8192 + sw128(i, jo + 8 * c8));
@@ -705,12 +735,16 @@ __global__ void __launch_bounds__(TC_THREADS, 1) chunk_tc_kernel(
           *reinterpret_cast<uint4*>(xu + sw128(i, jo + 8 * c8)) = pack8(vf);
         }
       }
+      // meanwhile rows 64..127 (the other two warps of each warpgroup): the previous chunk's
+      // output (its D_KS block and the P U rows stay valid until this chunk's step 3)
+      if (ok && ew >= 2 && c >= 1) write_out(c - 1, g_row_prev);
       TC_TS(12);
       fence_proxy_async_smem();
       TC_TS(13);
       tc_fence_before();
       if (!named_bar_and(1, TC_WORKERS, ok)) {
         fail(GDN_ERR_TIMEOUT);
+        all_ok = false;
         break;
       }
       TC_TS(2);
@@ -753,6 +787,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) chunk_tc_kernel(
       tc_fence_before();
       if (!named_bar_and(1, TC_WORKERS, ok)) {
         fail(GDN_ERR_TIMEOUT);
+        all_ok = false;
         break;
       }
       TC_TS(4);
@@ -777,26 +812,6 @@ __global__ void __launch_bounds__(TC_THREADS, 1) chunk_tc_kernel(
       // the [T'; P] buffer of this chunk has been read by both of its MMAs: hand it back
       if (leader && ok) mbar_arrive_peer(peer_addr(smem_u32(&bars[B_PREP_EMPTY0 + b]), 0));
       TC_TS(8);
-      if (ok && ew >= 2) {
-        // O = scale (Gamma_r (Q S0^T)_r + (P U)_r), rows r = i - 64
-        const int r = i - 64;
-        float qs[32], pu[32];
-        tmem_ld16(tmem + TM_KS + jb + lane_off, *reinterpret_cast<float(*)[16]>(qs));
-        tmem_ld16(tmem + TM_KS + jb + 16 + lane_off, *reinterpret_cast<float(*)[16]>(qs + 16));
-        tmem_ld16(tmem + TM_U + jb + lane_off, *reinterpret_cast<float(*)[16]>(pu));
-        tmem_ld16(tmem + TM_U + jb + 16 + lane_off, *reinterpret_cast<float(*)[16]>(pu + 16));
-        tmem_ld_wait();
-        if (r < L) {
-          __nv_bfloat16* orow = P.out + ((t0 + r) * P.Hv + h) * 128 + jb;
-#pragma unroll
-          for (int c8 = 0; c8 < 4; ++c8) {
-            float f[8];
-#pragma unroll
-            for (int q = 0; q < 8; ++q) f[q] = P.scale * fmaf(g_row, qs[8 * c8 + q], pu[8 * c8 + q]);
-            *reinterpret_cast<uint4*>(orow + 8 * c8) = pack8(f);
-          }
-        }
-      }
       TC_TS(9);
       if (ok) {
         float sv[32];
@@ -812,9 +827,15 @@ __global__ void __launch_bounds__(TC_THREADS, 1) chunk_tc_kernel(
       tc_fence_before();
       if (!named_bar_and(1, TC_WORKERS, ok)) {
         fail(GDN_ERR_TIMEOUT);
+        all_ok = false;
         break;
       }
+      g_row_prev = g_row;
       TC_TS(6);
+    }
+    if (all_ok && nchunks > 0 && ew >= 2) {
+      tc_fence_after();
+      write_out(nchunks - 1, g_row_prev);
     }
     TC_TRACE_FLUSH(leader ? 3 : 4);
     if (warp == 0) cp_async_wait_all();  // no gate copy may still be landing at exit
