@@ -6,18 +6,28 @@
 //   pre[t,c] = bias[c] + sum_{i<K} w[c,i] * x[t-(K-1)+i, c]        y = silu(pre)
 //   each group of `group` channels among the first n_l2 channels:  y[t,G] /= sqrt(|y[t,G]|^2 + eps)
 //
-// HBM-bound stencil: x is read once (plus a K-1 token halo per tile, served by L2) and y written
-// once.  Each thread owns 8 consecutive channels (one 16-byte bf16 transaction per token) and walks
-// a tile of TT tokens, keeping the last K-1 inputs in registers; a warp covers 256 contiguous
-// channels, so every token row is read as 512-byte coalesced segments.  The L2 norm of a head is a
-// shuffle reduction over the group's group/8 lanes.
+// HBM-bound stencil: x is read once (plus a K-1 token halo per block) and y written once.  Each
+// thread owns 8 consecutive channels (one 16-byte bf16 vector per token) and streams a long,
+// contiguous token range of them; a warp covers 256 contiguous channels, so every token row is
+// read and written as 512-byte coalesced segments.
+//
+// Memory-level parallelism comes from a private per-thread ring in shared memory: each thread
+// keeps DEPTH-1 tokens of its own channels in flight with cp.async (16-byte, L1-bypassing), and
+// waits only for the oldest one.  Because a thread reads back only the slots it filled itself,
+// no block-wide synchronisation is needed.  The last K-1 inputs live in registers as a circular
+// window whose rotation is unrolled, so no register moves are spent on shifting it.  The grid
+// is one wave (two blocks per SM for K <= 5), each block taking an equal share of the tokens of one
+// 2048-channel slab.  The L2 norm of a head is a shuffle reduction over the group's group/8
+// lanes, skipped by warps that hold only v channels.
 #include "gdn_internal.cuh"
 
 namespace gdn {
 
-constexpr int CONV_TT = 32;       // tokens per tile
-constexpr int CONV_THREADS = 128; // threads per block -> 1024 channels per block
-constexpr int CONV_U = 8;         // tokens loaded ahead per batch
+constexpr int CONV_THREADS = 256;     // 8 channels per thread -> 2048 channels per block
+// blocks per SM: two while weights + window fit the 128 registers that allows, else one
+__host__ __device__ constexpr int conv_blocks_per_sm(int K) { return K <= 5 ? 2 : 1; }
+constexpr int CONV_RING_BYTES = 256;  // per-thread ring: 16 bf16 tokens or 8 fp32 tokens
+constexpr int CONV_MIN_TOKENS = 64;   // fewest tokens per block
 
 __device__ __forceinline__ void seq_range(const int32_t* cu, int64_t T, int n, int64_t& s,
                                           int64_t& e) {
@@ -30,16 +40,66 @@ __device__ __forceinline__ void seq_range(const int32_t* cu, int64_t T, int n, i
   }
 }
 
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+__device__ __forceinline__ uint4 lds128(uint32_t a) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "r"(a)
+               : "memory");
+  return v;
+}
+
+// 8 channels of one token, as stored in the ring (V 16-byte parts, each CONV_THREADS*16 apart)
+__device__ __forceinline__ void ring_to_float(uint32_t a, const __nv_bfloat16*, float (&f)[8]) {
+  const uint4 u = lds128(a);
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    f[2 * i] = __uint_as_float(w[i] << 16);
+    f[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+  }
+}
+__device__ __forceinline__ void ring_to_float(uint32_t a, const float*, float (&f)[8]) {
+  const uint4 u = lds128(a);
+  const uint4 v = lds128(a + CONV_THREADS * 16);
+  f[0] = __uint_as_float(u.x); f[1] = __uint_as_float(u.y);
+  f[2] = __uint_as_float(u.z); f[3] = __uint_as_float(u.w);
+  f[4] = __uint_as_float(v.x); f[5] = __uint_as_float(v.y);
+  f[6] = __uint_as_float(v.z); f[7] = __uint_as_float(v.w);
+}
+
 template <typename T, int K>
-__global__ void __launch_bounds__(CONV_THREADS, 4) conv_silu_kernel(
+__global__ void __launch_bounds__(CONV_THREADS, conv_blocks_per_sm(K)) conv_silu_kernel(
     const T* __restrict__ x, const float* __restrict__ w, const float* __restrict__ bias,
     int64_t n_tok, int64_t Tlen, int C, const int32_t* __restrict__ cu, int N, int n_l2,
     int group, float l2_eps, const float* __restrict__ cs_in, float* __restrict__ cs_out,
     T* __restrict__ y) {
+  constexpr int V = (int)sizeof(T) / 2;              // 16-byte parts per 8-channel vector
+  constexpr int DEPTH = CONV_RING_BYTES / (16 * V);  // ring slots per thread
+  constexpr uint32_t SLOT = V * CONV_THREADS * 16;   // bytes per ring slot (whole block)
+  constexpr int W = K > 1 ? K - 1 : 1;               // window length
+  constexpr int U = W >= 4 ? W : W * (8 / W);        // tokens per unrolled group (multiple of W)
+  static_assert((DEPTH & (DEPTH - 1)) == 0, "ring depth must be a power of two");
+  extern __shared__ __align__(16) uint4 conv_ring[];
+
   const int cc = blockIdx.y * CONV_THREADS + threadIdx.x;
   const int c0 = cc * 8;
+  const int warp_c0 = (blockIdx.y * CONV_THREADS + (threadIdx.x & ~31)) * 8;
+  if (warp_c0 >= C) return;  // whole warp past the last channel (warp-uniform)
   const bool chan_ok = c0 < C;
   const bool do_norm = chan_ok && c0 < n_l2;
+  const int lanes_per_group = group >> 3;  // 0 when no normalisation
+  const bool warp_norm = lanes_per_group > 0 && warp_c0 < n_l2;
 
   float wt[8][K];
   float bs[8];
@@ -50,7 +110,7 @@ __global__ void __launch_bounds__(CONV_THREADS, 4) conv_silu_kernel(
     for (int i = 0; i < K; ++i) wt[e][i] = chan_ok ? __ldg(w + (int64_t)(c0 + e) * K + i) : 0.0f;
   }
 
-  // Zero-length sequences still produce a conv state (copied through); tile 0 handles them.
+  // Zero-length sequences still produce a conv state (copied through); blocks of column 0 do it.
   if (blockIdx.x == 0 && cs_out && chan_ok && cu) {
     for (int n = 0; n < N; ++n) {
       if (cu[n + 1] != cu[n]) continue;
@@ -62,16 +122,48 @@ __global__ void __launch_bounds__(CONV_THREADS, 4) conv_silu_kernel(
     }
   }
 
-  const int64_t t_begin = (int64_t)blockIdx.x * CONV_TT;
-  if (t_begin >= n_tok) return;
-  const int64_t t_end = min(t_begin + (int64_t)CONV_TT, n_tok);
+  const int64_t t_begin = n_tok * blockIdx.x / gridDim.x;
+  const int64_t t_end = n_tok * (blockIdx.x + 1) / gridDim.x;
+  if (t_begin >= t_end) return;  // block-uniform
+
+  // ---- per-thread cp.async ring: token t_begin + i lives in slot i % DEPTH
+  const uint32_t ring = (uint32_t)__cvta_generic_to_shared(conv_ring) + threadIdx.x * 16u;
+  const T* xsrc = x + c0;
+  auto issue = [&](int64_t i) {  // start loading token t_begin + i; one commit group per token
+    const int64_t t = t_begin + i;
+    if (chan_ok && t < t_end) {
+      const uint32_t dst = ring + (uint32_t)(i & (DEPTH - 1)) * SLOT;
+      const char* src = reinterpret_cast<const char*>(xsrc + t * C);
+#pragma unroll
+      for (int v = 0; v < V; ++v) cp_async16(dst + v * CONV_THREADS * 16, src + 16 * v);
+    }
+    cp_async_commit();
+  };
+  // Token t_begin + i: refill the slot consumed by the previous token (its value is already in
+  // registers and used), wait for the oldest load, read it back.
+  auto take = [&](int64_t i, float (&xt)[8]) {
+    issue(i + DEPTH - 1);
+    cp_async_wait<DEPTH - 1>();
+    if (chan_ok) {
+      ring_to_float(ring + (uint32_t)(i & (DEPTH - 1)) * SLOT, x, xt);
+    } else {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) xt[e] = 0.0f;
+    }
+  };
+#pragma unroll 1
+  for (int i = 0; i < DEPTH - 1; ++i) issue(i);
 
   int n = seq_of_token(cu, N, Tlen, t_begin);
   int64_t s_beg, s_end;
   seq_range(cu, Tlen, n, s_beg, s_end);
 
-  // win[j][e]: input at position t-(K-1)+j for the next token t (oldest first).
-  float win[K > 1 ? K - 1 : 1][8];
+  // win[j][e], j = 0..K-2, in "phase 0" order: oldest input first.
+  float win[W][8];
+#pragma unroll
+  for (int j = 0; j < W; ++j)
+#pragma unroll
+    for (int e = 0; e < 8; ++e) win[j][e] = 0.0f;
   auto fill_window = [&](int64_t t) {
 #pragma unroll
     for (int j = 0; j < K - 1; ++j) {
@@ -93,74 +185,119 @@ __global__ void __launch_bounds__(CONV_THREADS, 4) conv_silu_kernel(
       }
     }
   };
-  fill_window(t_begin);
 
-  const int lanes_per_group = group >> 3;  // 0 when no normalisation
-  for (int64_t tb = t_begin; tb < t_end; tb += CONV_U) {
-    Raw8<T> xs[CONV_U];
+  // conv + SiLU + (optional) head L2 norm + store of one token whose window order is rotated by
+  // `ph` (the oldest input sits in win[ph]); the oldest slot is then overwritten with xt.
+  auto token = [&](int64_t t, const float (&xt)[8], int ph) {
+    float acc[8];
 #pragma unroll
-    for (int u = 0; u < CONV_U; ++u) {
-      if (chan_ok && tb + u < t_end)
-        xs[u].load(x + (tb + u) * C + c0);
-      else
-        xs[u].zero();
+    for (int e = 0; e < 8; ++e) {
+      float a = bs[e];
+#pragma unroll
+      for (int j = 0; j < K - 1; ++j) a = fmaf(wt[e][j], win[(ph + j) % W][e], a);
+      acc[e] = silu_fast(fmaf(wt[e][K - 1], xt[e], a));
     }
+    if (K > 1) {
 #pragma unroll
-    for (int u = 0; u < CONV_U; ++u) {
-      const int64_t t = tb + u;
-      if (t >= t_end) break;  // uniform across the block
-      if (t >= s_end) {       // entered the next non-empty sequence
-        if (cu) {
-          while (n + 1 < N && (int64_t)cu[n + 1] <= t) ++n;
-        } else {
-          n = (int)(t / Tlen);
-        }
-        seq_range(cu, Tlen, n, s_beg, s_end);
-        fill_window(t);
+      for (int e = 0; e < 8; ++e) win[ph][e] = xt[e];
+    }
+    if (warp_norm) {
+      float ss = 0.0f;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) ss = fmaf(acc[e], acc[e], ss);
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1)
+        if (o < lanes_per_group) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+      const float inv = do_norm ? rsqrtf(ss + l2_eps) : 1.0f;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) acc[e] *= inv;
+    }
+    if (chan_ok) store8(y + t * C + c0, acc);
+  };
+
+  int64_t t = t_begin;
+  if (t >= s_beg && t < s_end) fill_window(t);
+  while (t < t_end) {
+    if (t >= s_end) {  // entered the next non-empty sequence
+      if (cu) {
+        while (n + 1 < N && (int64_t)cu[n + 1] <= t) ++n;
+      } else {
+        n = (int)(t / Tlen);
       }
-      // false only when cu_seqlens is malformed (token outside every sequence): skip writes
-      const bool tok_ok = t >= s_beg && t < s_end;
+      seq_range(cu, Tlen, n, s_beg, s_end);
+      if (t >= s_beg && t < s_end) fill_window(t);
+    }
+    if (t < s_beg || t >= s_end) {
+      // token outside every sequence (only a malformed cu_seqlens): consume it, write nothing
+      const int64_t stop = t < s_beg ? min(s_beg, t_end) : t_end;
+      for (; t < stop; ++t) {
+        float xt[8];
+        take(t - t_begin, xt);
+      }
+      continue;
+    }
+    const int64_t seg_end = min(s_end, t_end);
+    // groups of U tokens: the window rotates through all W phases and returns to phase 0
+    while (t + U <= seg_end) {
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        float xt[8];
+        take(t + u - t_begin, xt);
+        token(t + u, xt, u % W);
+      }
+      t += U;
+    }
+    // tail: phase 0 every token, window shifted in registers
+    for (; t < seg_end; ++t) {
       float xt[8];
-      xs[u].to_float(xt);
-      float acc[8];
+      take(t - t_begin, xt);
+      token(t, xt, 0);  // overwrote win[0] (the oldest) with xt: rotate back to phase 0
+      if (K > 2) {
+        float tmp[8];
 #pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        float a = bs[e];
+        for (int e = 0; e < 8; ++e) tmp[e] = win[0][e];
 #pragma unroll
-        for (int j = 0; j < K - 1; ++j) a = fmaf(wt[e][j], win[j][e], a);
-        acc[e] = silu_fast(fmaf(wt[e][K - 1], xt[e], a));
+        for (int j = 0; j + 1 < K - 1; ++j)
+#pragma unroll
+          for (int e = 0; e < 8; ++e) win[j][e] = win[j + 1][e];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) win[W - 1][e] = tmp[e];
       }
+    }
+    if (t == s_end && cs_out && chan_ok) {
+      // last token of sequence n was t-1: the window holds its last K-1 inputs, oldest first
 #pragma unroll
-      for (int j = 0; j + 1 < K - 1; ++j)
+      for (int e = 0; e < 8; ++e)
 #pragma unroll
-        for (int e = 0; e < 8; ++e) win[j][e] = win[j + 1][e];
-      if (K > 1) {
-#pragma unroll
-        for (int e = 0; e < 8; ++e) win[K > 1 ? K - 2 : 0][e] = xt[e];
-      }
-      if (lanes_per_group) {
-        float ss = 0.0f;
-#pragma unroll
-        for (int e = 0; e < 8; ++e) ss = fmaf(acc[e], acc[e], ss);
-        for (int o = lanes_per_group >> 1; o > 0; o >>= 1)
-          ss += __shfl_xor_sync(0xffffffffu, ss, o);
-        if (do_norm) {
-          const float inv = rsqrtf(ss + l2_eps);
-#pragma unroll
-          for (int e = 0; e < 8; ++e) acc[e] *= inv;
-        }
-      }
-      if (chan_ok && tok_ok) store8(y + t * C + c0, acc);
-      if (cs_out && chan_ok && tok_ok && t == s_end - 1) {
-        // last token of sequence n: the window now holds its last K-1 inputs
-#pragma unroll
-        for (int e = 0; e < 8; ++e)
-#pragma unroll
-          for (int j = 0; j < K - 1; ++j)
-            cs_out[((int64_t)n * C + c0 + e) * (K - 1) + j] = win[j][e];
-      }
+        for (int j = 0; j < K - 1; ++j)
+          cs_out[((int64_t)n * C + c0 + e) * (K - 1) + j] = win[j][e];
     }
   }
+  cp_async_wait<0>();  // leave no copy in flight into shared memory
+}
+
+template <typename T, int K>
+static cudaError_t launch_conv_k(int sms, int64_t n_tok, int slabs, const T* x, const float* w, const float* bias,
+                                 int64_t T_, int C, const int32_t* cu, int N, int n_l2, int group,
+                                 float l2_eps, const float* cs_in, float* cs_out, T* y,
+                                 cudaStream_t s) {
+  // one wave: every resident block slot gets an equal share of one slab's tokens
+  int64_t cols = ((int64_t)sms * conv_blocks_per_sm(K) + slabs - 1) / slabs;
+  const int64_t by_len = (n_tok + CONV_MIN_TOKENS - 1) / CONV_MIN_TOKENS;
+  if (cols > by_len) cols = by_len;
+  if (cols < 1) cols = 1;
+  const dim3 grid((unsigned)cols, (unsigned)slabs);
+  constexpr int smem = CONV_RING_BYTES * CONV_THREADS;
+  static bool attr_set = false;  // idempotent attribute; a benign race between host threads
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(conv_silu_kernel<T, K>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  conv_silu_kernel<T, K><<<grid, CONV_THREADS, smem, s>>>(x, w, bias, n_tok, T_, C, cu, N, n_l2,
+                                                          group, l2_eps, cs_in, cs_out, y);
+  return cudaGetLastError();
 }
 
 template <typename T>
@@ -168,18 +305,17 @@ static cudaError_t launch_conv_t(const T* x, const float* w, const float* bias, 
                                  int C, int K, const int32_t* cu, int N, int n_l2, int group,
                                  float l2_eps, const float* cs_in, float* cs_out, T* y,
                                  cudaStream_t s) {
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int64_t n_tok = (int64_t)B * T_;
-  const int64_t tiles = n_tok > 0 ? (n_tok + CONV_TT - 1) / CONV_TT : 1;
-  const int chunks = C / 8;
-  dim3 grid((unsigned)tiles, (unsigned)((chunks + CONV_THREADS - 1) / CONV_THREADS));
-  if (grid.y > 65535u) return cudaErrorInvalidConfiguration;
+  const int slabs = (C / 8 + CONV_THREADS - 1) / CONV_THREADS;
+  if (slabs > 65535) return cudaErrorInvalidConfiguration;
   switch (K) {
-#define GDN_CONV_CASE(KK)                                                                     \
-  case KK:                                                                                    \
-    conv_silu_kernel<T, KK><<<grid, CONV_THREADS, 0, s>>>(x, w, bias, n_tok, T_, C, cu, N,    \
-                                                          n_l2, group, l2_eps, cs_in, cs_out, \
-                                                          y);                                 \
-    break;
+#define GDN_CONV_CASE(KK) \
+  case KK:                \
+    return launch_conv_k<T, KK>(sms, n_tok, slabs, x, w, bias, T_, C, cu, N, n_l2, group, \
+                                l2_eps, cs_in, cs_out, y, s);
     GDN_CONV_CASE(1)
     GDN_CONV_CASE(2)
     GDN_CONV_CASE(3)
@@ -191,7 +327,6 @@ static cudaError_t launch_conv_t(const T* x, const float* w, const float* bias, 
 #undef GDN_CONV_CASE
     default: return cudaErrorInvalidValue;
   }
-  return cudaGetLastError();
 }
 
 cudaError_t launch_conv(const void* x, gdn_dtype dt, const float* w, const float* bias, int B,
