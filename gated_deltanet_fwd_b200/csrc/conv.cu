@@ -12,20 +12,24 @@
 // read and written as 512-byte coalesced segments.
 //
 // Memory-level parallelism comes from a private per-thread ring in shared memory: each thread
-// keeps DEPTH-1 tokens of its own channels in flight with cp.async (16-byte, L1-bypassing), and
-// waits only for the oldest one.  Because a thread reads back only the slots it filled itself,
+// keeps DEPTH-2 tokens of its own channels in flight with cp.async (16-byte, L1-bypassing), and
+// waits only for the oldest ones.  Because a thread reads back only the slots it filled itself,
 // no block-wide synchronisation is needed.  The last K-1 inputs live in registers as a circular
-// window whose rotation is unrolled, so no register moves are spent on shifting it.  The grid
-// is one wave (two blocks per SM for K <= 5), each block taking an equal share of the tokens of one
+// window whose rotation is unrolled, so no register moves are spent on shifting it, and tokens
+// are computed two at a time in packed fp32 (two lanes per instruction) so that the latency
+// chains of conv -> SiLU -> norm overlap.  The grid
+// is one wave (two blocks per SM for K <= 4), each block taking an equal share of the tokens of one
 // 2048-channel slab.  The L2 norm of a head is a shuffle reduction over the group's group/8
 // lanes, skipped by warps that hold only v channels.
+#include <type_traits>
+
 #include "gdn_internal.cuh"
 
 namespace gdn {
 
 constexpr int CONV_THREADS = 256;     // 8 channels per thread -> 2048 channels per block
-// blocks per SM: two while weights + window fit the 128 registers that allows, else one
-__host__ __device__ constexpr int conv_blocks_per_sm(int K) { return K <= 5 ? 2 : 1; }
+// blocks per SM: two while weights + window fit the 128 registers that allows (K <= 4), else one
+__host__ __device__ constexpr int conv_blocks_per_sm(int K) { return K <= 4 ? 2 : 1; }
 constexpr int CONV_RING_BYTES = 256;  // per-thread ring: 16 bf16 tokens or 8 fp32 tokens
 constexpr int CONV_MIN_TOKENS = 64;   // fewest tokens per block
 
@@ -59,23 +63,51 @@ __device__ __forceinline__ uint4 lds128(uint32_t a) {
   return v;
 }
 
-// 8 channels of one token, as stored in the ring (V 16-byte parts, each CONV_THREADS*16 apart)
-__device__ __forceinline__ void ring_to_float(uint32_t a, const __nv_bfloat16*, float (&f)[8]) {
+// 8 channels of one token, as stored in the ring (V 16-byte parts, CONV_THREADS*16 apart), as
+// four channel pairs
+__device__ __forceinline__ void ring_to_float2(uint32_t a, const __nv_bfloat16*, float2 (&f)[4]) {
   const uint4 u = lds128(a);
   const uint32_t w[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    f[2 * i] = __uint_as_float(w[i] << 16);
-    f[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
-  }
+  for (int i = 0; i < 4; ++i)
+    f[i] = make_float2(__uint_as_float(w[i] << 16), __uint_as_float(w[i] & 0xffff0000u));
 }
-__device__ __forceinline__ void ring_to_float(uint32_t a, const float*, float (&f)[8]) {
+__device__ __forceinline__ void ring_to_float2(uint32_t a, const float*, float2 (&f)[4]) {
   const uint4 u = lds128(a);
   const uint4 v = lds128(a + CONV_THREADS * 16);
-  f[0] = __uint_as_float(u.x); f[1] = __uint_as_float(u.y);
-  f[2] = __uint_as_float(u.z); f[3] = __uint_as_float(u.w);
-  f[4] = __uint_as_float(v.x); f[5] = __uint_as_float(v.y);
-  f[6] = __uint_as_float(v.z); f[7] = __uint_as_float(v.w);
+  f[0] = make_float2(__uint_as_float(u.x), __uint_as_float(u.y));
+  f[1] = make_float2(__uint_as_float(u.z), __uint_as_float(u.w));
+  f[2] = make_float2(__uint_as_float(v.x), __uint_as_float(v.y));
+  f[3] = make_float2(__uint_as_float(v.z), __uint_as_float(v.w));
+}
+__device__ __forceinline__ void store8x2(__nv_bfloat16* p, const float2 (&f)[4]) {
+  uint4 u;
+  __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&u);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) h[i] = __float22bfloat162_rn(f[i]);
+  *reinterpret_cast<uint4*>(p) = u;
+}
+__device__ __forceinline__ void store8x2(float* p, const float2 (&f)[4]) {
+  reinterpret_cast<float4*>(p)[0] = make_float4(f[0].x, f[0].y, f[1].x, f[1].y);
+  reinterpret_cast<float4*>(p)[1] = make_float4(f[2].x, f[2].y, f[3].x, f[3].y);
+}
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+__device__ __forceinline__ float rcp_approx(float x) {
+  float y;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+// silu on a channel pair: x * 1 / (1 + 2^(-x log2 e)); the packed fp32 ops (two lanes per
+// instruction) halve the FMA-pipe work, the two special-function ops per element remain.  At
+// x -> -inf the exponential overflows to +inf and the result is -0, the correct limit.
+__device__ __forceinline__ float2 silu2(float2 x) {
+  const float2 m = __fmul2_rn(x, make_float2(-1.4426950408889634f, -1.4426950408889634f));
+  const float2 d = __fadd2_rn(make_float2(ex2_approx(m.x), ex2_approx(m.y)), make_float2(1.f, 1.f));
+  return __fmul2_rn(x, make_float2(rcp_approx(d.x), rcp_approx(d.y)));
 }
 
 template <typename T, int K>
@@ -88,7 +120,9 @@ __global__ void __launch_bounds__(CONV_THREADS, conv_blocks_per_sm(K)) conv_silu
   constexpr int DEPTH = CONV_RING_BYTES / (16 * V);  // ring slots per thread
   constexpr uint32_t SLOT = V * CONV_THREADS * 16;   // bytes per ring slot (whole block)
   constexpr int W = K > 1 ? K - 1 : 1;               // window length
-  constexpr int U = W >= 4 ? W : W * (8 / W);        // tokens per unrolled group (multiple of W)
+  // tokens per unrolled group: a multiple of W (the window returns to phase 0) and of 2 (tokens
+  // go in pairs)
+  constexpr int U = W >= 4 ? (W % 2 ? 2 * W : W) : W * (8 / W);
   static_assert((DEPTH & (DEPTH - 1)) == 0, "ring depth must be a power of two");
   extern __shared__ __align__(16) uint4 conv_ring[];
 
@@ -101,13 +135,18 @@ __global__ void __launch_bounds__(CONV_THREADS, conv_blocks_per_sm(K)) conv_silu
   const int lanes_per_group = group >> 3;  // 0 when no normalisation
   const bool warp_norm = lanes_per_group > 0 && warp_c0 < n_l2;
 
-  float wt[8][K];
-  float bs[8];
+  // weights and bias of the thread's 8 channels, as channel pairs (p: channels 2p, 2p+1)
+  float2 wt[4][K];
+  float2 bs[4];
 #pragma unroll
-  for (int e = 0; e < 8; ++e) {
-    bs[e] = (chan_ok && bias) ? __ldg(bias + c0 + e) : 0.0f;
+  for (int p = 0; p < 4; ++p) {
+    bs[p] = (chan_ok && bias) ? make_float2(__ldg(bias + c0 + 2 * p), __ldg(bias + c0 + 2 * p + 1))
+                              : make_float2(0.f, 0.f);
 #pragma unroll
-    for (int i = 0; i < K; ++i) wt[e][i] = chan_ok ? __ldg(w + (int64_t)(c0 + e) * K + i) : 0.0f;
+    for (int i = 0; i < K; ++i)
+      wt[p][i] = chan_ok ? make_float2(__ldg(w + (int64_t)(c0 + 2 * p) * K + i),
+                                       __ldg(w + (int64_t)(c0 + 2 * p + 1) * K + i))
+                         : make_float2(0.f, 0.f);
   }
 
   // Zero-length sequences still produce a conv state (copied through); blocks of column 0 do it.
@@ -139,81 +178,116 @@ __global__ void __launch_bounds__(CONV_THREADS, conv_blocks_per_sm(K)) conv_silu
     }
     cp_async_commit();
   };
-  // Token t_begin + i: refill the slot consumed by the previous token (its value is already in
-  // registers and used), wait for the oldest load, read it back.
-  auto take = [&](int64_t i, float (&xt)[8]) {
-    issue(i + DEPTH - 1);
-    cp_async_wait<DEPTH - 1>();
-    if (chan_ok) {
-      ring_to_float(ring + (uint32_t)(i & (DEPTH - 1)) * SLOT, x, xt);
-    } else {
+  // Before token t_begin + i is taken, tokens up to i + DEPTH - 3 have been issued.  Taking
+  // NT (1 or 2) tokens refills the NT slots consumed by the previous step (their values are
+  // already in registers and used), then waits until token i + NT - 1 has landed: DEPTH - 2
+  // newer groups may still be in flight.
+  auto take = [&](auto nt, int64_t i, float2 (*xt)[4]) {
+    constexpr int NT = decltype(nt)::value;
 #pragma unroll
-      for (int e = 0; e < 8; ++e) xt[e] = 0.0f;
+    for (int k = 0; k < NT; ++k) issue(i + k + DEPTH - 2);
+    cp_async_wait<DEPTH - 2>();
+#pragma unroll
+    for (int k = 0; k < NT; ++k) {
+      if (chan_ok) {
+        ring_to_float2(ring + (uint32_t)((i + k) & (DEPTH - 1)) * SLOT, x, xt[k]);
+      } else {
+#pragma unroll
+        for (int p = 0; p < 4; ++p) xt[k][p] = make_float2(0.f, 0.f);
+      }
     }
   };
 #pragma unroll 1
-  for (int i = 0; i < DEPTH - 1; ++i) issue(i);
+  for (int i = 0; i < DEPTH - 2; ++i) issue(i);
 
   int n = seq_of_token(cu, N, Tlen, t_begin);
   int64_t s_beg, s_end;
   seq_range(cu, Tlen, n, s_beg, s_end);
 
-  // win[j][e], j = 0..K-2, in "phase 0" order: oldest input first.
-  float win[W][8];
+  // win[j][q], j = 0..K-2, in "phase 0" order: oldest input first; q = channel pair.
+  float2 win[W][4];
 #pragma unroll
   for (int j = 0; j < W; ++j)
 #pragma unroll
-    for (int e = 0; e < 8; ++e) win[j][e] = 0.0f;
+    for (int q = 0; q < 4; ++q) win[j][q] = make_float2(0.f, 0.f);
   auto fill_window = [&](int64_t t) {
 #pragma unroll
     for (int j = 0; j < K - 1; ++j) {
       const int64_t p = t - (K - 1) + j;
+      float f[8];
       if (!chan_ok) {
 #pragma unroll
-        for (int e = 0; e < 8; ++e) win[j][e] = 0.0f;
+        for (int e = 0; e < 8; ++e) f[e] = 0.0f;
       } else if (p >= s_beg && p >= 0 && p < n_tok) {
-        load8(x + p * C + c0, win[j]);
+        load8(x + p * C + c0, f);
       } else {
         // before the sequence start: carried conv state (or zero).  The range check only
         // matters for a malformed cu_seqlens, which must not cause out-of-bounds reads.
         const int64_t r = (K - 1) + (p - s_beg);
 #pragma unroll
         for (int e = 0; e < 8; ++e)
-          win[j][e] = (cs_in && r >= 0 && r < K - 1)
-                          ? cs_in[((int64_t)n * C + c0 + e) * (K - 1) + r]
-                          : 0.0f;
+          f[e] = (cs_in && r >= 0 && r < K - 1) ? cs_in[((int64_t)n * C + c0 + e) * (K - 1) + r]
+                                                : 0.0f;
       }
+#pragma unroll
+      for (int q = 0; q < 4; ++q) win[j][q] = make_float2(f[2 * q], f[2 * q + 1]);
     }
   };
 
-  // conv + SiLU + (optional) head L2 norm + store of one token whose window order is rotated by
-  // `ph` (the oldest input sits in win[ph]); the oldest slot is then overwritten with xt.
-  auto token = [&](int64_t t, const float (&xt)[8], int ph) {
-    float acc[8];
+  // conv + SiLU + (optional) head L2 norm + store of NT consecutive tokens from t.  The window
+  // order is rotated by `ph` (token t's oldest input sits in win[ph]); each token overwrites its
+  // oldest slot with its own input, which the next token then sees as its newest.  Two tokens
+  // are computed side by side, so their dependency chains overlap.
+  auto tokens = [&](auto nt, int64_t t, const float2 (*xt)[4], int ph) {
+    constexpr int NT = decltype(nt)::value;
+    float2 acc[NT][4];
 #pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      float a = bs[e];
+    for (int k = 0; k < NT; ++k) {
 #pragma unroll
-      for (int j = 0; j < K - 1; ++j) a = fmaf(wt[e][j], win[(ph + j) % W][e], a);
-      acc[e] = silu_fast(fmaf(wt[e][K - 1], xt[e], a));
+      for (int q = 0; q < 4; ++q) {
+        float2 a = bs[q];
+#pragma unroll
+        for (int j = 0; j < K - 1; ++j) a = __ffma2_rn(wt[q][j], win[(ph + k + j) % W][q], a);
+        acc[k][q] = __ffma2_rn(wt[q][K - 1], xt[k][q], a);
+      }
+      if (K > 1) {
+#pragma unroll
+        for (int q = 0; q < 4; ++q) win[(ph + k) % W][q] = xt[k][q];
+      }
     }
-    if (K > 1) {
 #pragma unroll
-      for (int e = 0; e < 8; ++e) win[ph][e] = xt[e];
-    }
+    for (int k = 0; k < NT; ++k)
+#pragma unroll
+      for (int q = 0; q < 4; ++q) acc[k][q] = silu2(acc[k][q]);
     if (warp_norm) {
-      float ss = 0.0f;
+      float ss[NT];
 #pragma unroll
-      for (int e = 0; e < 8; ++e) ss = fmaf(acc[e], acc[e], ss);
+      for (int k = 0; k < NT; ++k) {
+        float2 s2 = __fmul2_rn(acc[k][0], acc[k][0]);
+#pragma unroll
+        for (int q = 1; q < 4; ++q) s2 = __ffma2_rn(acc[k][q], acc[k][q], s2);
+        ss[k] = s2.x + s2.y;
+      }
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1)
-        if (o < lanes_per_group) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-      const float inv = do_norm ? rsqrtf(ss + l2_eps) : 1.0f;
+        if (o < lanes_per_group) {
 #pragma unroll
-      for (int e = 0; e < 8; ++e) acc[e] *= inv;
+          for (int k = 0; k < NT; ++k) ss[k] += __shfl_xor_sync(0xffffffffu, ss[k], o);
+        }
+#pragma unroll
+      for (int k = 0; k < NT; ++k) {
+        const float inv = do_norm ? rsqrtf(ss[k] + l2_eps) : 1.0f;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) acc[k][q] = __fmul2_rn(acc[k][q], make_float2(inv, inv));
+      }
     }
-    if (chan_ok) store8(y + t * C + c0, acc);
+    if (chan_ok) {
+#pragma unroll
+      for (int k = 0; k < NT; ++k) store8x2(y + (t + k) * C + c0, acc[k]);
+    }
   };
+  using One = std::integral_constant<int, 1>;
+  using Two = std::integral_constant<int, 2>;
 
   int64_t t = t_begin;
   if (t >= s_beg && t < s_end) fill_window(t);
@@ -231,8 +305,8 @@ __global__ void __launch_bounds__(CONV_THREADS, conv_blocks_per_sm(K)) conv_silu
       // token outside every sequence (only a malformed cu_seqlens): consume it, write nothing
       const int64_t stop = t < s_beg ? min(s_beg, t_end) : t_end;
       for (; t < stop; ++t) {
-        float xt[8];
-        take(t - t_begin, xt);
+        float2 xt[1][4];
+        take(One{}, t - t_begin, xt);
       }
       continue;
     }
@@ -240,37 +314,39 @@ __global__ void __launch_bounds__(CONV_THREADS, conv_blocks_per_sm(K)) conv_silu
     // groups of U tokens: the window rotates through all W phases and returns to phase 0
     while (t + U <= seg_end) {
 #pragma unroll
-      for (int u = 0; u < U; ++u) {
-        float xt[8];
-        take(t + u - t_begin, xt);
-        token(t + u, xt, u % W);
+      for (int u = 0; u < U; u += 2) {
+        float2 xt[2][4];
+        take(Two{}, t + u - t_begin, xt);
+        tokens(Two{}, t + u, xt, u % W);
       }
       t += U;
     }
     // tail: phase 0 every token, window shifted in registers
     for (; t < seg_end; ++t) {
-      float xt[8];
-      take(t - t_begin, xt);
-      token(t, xt, 0);  // overwrote win[0] (the oldest) with xt: rotate back to phase 0
+      float2 xt[1][4];
+      take(One{}, t - t_begin, xt);
+      tokens(One{}, t, xt, 0);  // overwrote win[0] (the oldest) with xt: rotate back to phase 0
       if (K > 2) {
-        float tmp[8];
+        float2 tmp[4];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) tmp[e] = win[0][e];
+        for (int q = 0; q < 4; ++q) tmp[q] = win[0][q];
 #pragma unroll
         for (int j = 0; j + 1 < K - 1; ++j)
 #pragma unroll
-          for (int e = 0; e < 8; ++e) win[j][e] = win[j + 1][e];
+          for (int q = 0; q < 4; ++q) win[j][q] = win[j + 1][q];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) win[W - 1][e] = tmp[e];
+        for (int q = 0; q < 4; ++q) win[W - 1][q] = tmp[q];
       }
     }
     if (t == s_end && cs_out && chan_ok) {
       // last token of sequence n was t-1: the window holds its last K-1 inputs, oldest first
 #pragma unroll
-      for (int e = 0; e < 8; ++e)
+      for (int q = 0; q < 4; ++q)
 #pragma unroll
-        for (int j = 0; j < K - 1; ++j)
-          cs_out[((int64_t)n * C + c0 + e) * (K - 1) + j] = win[j][e];
+        for (int j = 0; j < K - 1; ++j) {
+          cs_out[((int64_t)n * C + c0 + 2 * q) * (K - 1) + j] = win[j][q].x;
+          cs_out[((int64_t)n * C + c0 + 2 * q + 1) * (K - 1) + j] = win[j][q].y;
+        }
     }
   }
   cp_async_wait<0>();  // leave no copy in flight into shared memory
