@@ -8,13 +8,15 @@
 //
 // HBM-bound: reads x and z, writes y, each once (3 * dim * elem bytes per row).  dim / 8 threads
 // share a row (8 elements = one 16-byte bf16 transaction each); the row's sum of squares is a
-// shuffle reduction inside that lane group.
+// shuffle reduction inside that lane group.  Each thread keeps RMS_U rows' loads in flight.
 #include "gdn_internal.cuh"
 
 namespace gdn {
 
+constexpr int RMS_U = 4;  // rows in flight per thread
+
 template <typename T, int TPR>
-__global__ void __launch_bounds__(256) rmsnorm_gated_kernel(const T* __restrict__ x,
+__global__ void __launch_bounds__(256, 4) rmsnorm_gated_kernel(const T* __restrict__ x,
                                                             const T* __restrict__ z,
                                                             const float* __restrict__ w,
                                                             float eps, int64_t rows,
@@ -22,29 +24,43 @@ __global__ void __launch_bounds__(256) rmsnorm_gated_kernel(const T* __restrict_
   constexpr int DIM = TPR * 8;
   constexpr int ROWS_PER_BLOCK = 256 / TPR;
   const int sub = threadIdx.x % TPR;
-  const int64_t row0 = (int64_t)blockIdx.x * ROWS_PER_BLOCK + threadIdx.x / TPR;
+  const int rsub = threadIdx.x / TPR;
   float wv[8];
 #pragma unroll
   for (int i = 0; i < 8; ++i) wv[i] = 1.0f + __ldg(w + sub * 8 + i);
   const int64_t rstride = (int64_t)gridDim.x * ROWS_PER_BLOCK;
-  for (int64_t r = row0; r - threadIdx.x / TPR < rows; r += rstride) {
-    const bool live = r < rows;
-    float xv[8], zv[8];
-    float ss = 0.0f;
-    if (live) {
-      load8(x + r * DIM + sub * 8, xv);
-      load8(z + r * DIM + sub * 8, zv);
+  // RMS_U rows per thread per pass: all their loads are issued before any is used
+  for (int64_t rb = (int64_t)blockIdx.x * ROWS_PER_BLOCK; rb < rows; rb += RMS_U * rstride) {
+    Raw8<T> xr[RMS_U], zr[RMS_U];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) ss = fmaf(xv[i], xv[i], ss);
+    for (int u = 0; u < RMS_U; ++u) {
+      const int64_t r = rb + u * rstride + rsub;
+      if (r < rows) {
+        xr[u].load(x + r * DIM + sub * 8);
+        zr[u].load(z + r * DIM + sub * 8);
+      } else {
+        xr[u].zero();
+        zr[u].zero();
+      }
     }
 #pragma unroll
-    for (int o = TPR / 2; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-    if (live) {
-      const float inv = rsqrtf(ss * (1.0f / DIM) + eps);
-      float yv[8];
+    for (int u = 0; u < RMS_U; ++u) {
+      const int64_t r = rb + u * rstride + rsub;
+      float xv[8], zv[8];
+      xr[u].to_float(xv);
+      zr[u].to_float(zv);
+      float ss = 0.0f;
 #pragma unroll
-      for (int i = 0; i < 8; ++i) yv[i] = xv[i] * inv * wv[i] * silu_fast(zv[i]);
-      store8(y + r * DIM + sub * 8, yv);
+      for (int i = 0; i < 8; ++i) ss = fmaf(xv[i], xv[i], ss);
+#pragma unroll
+      for (int o = TPR / 2; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+      if (r < rows) {
+        const float inv = rsqrtf(ss * (1.0f / DIM) + eps);
+        float yv[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) yv[i] = xv[i] * inv * wv[i] * silu_fast(zv[i]);
+        store8(y + r * DIM + sub * 8, yv);
+      }
     }
   }
 }
@@ -57,12 +73,19 @@ static cudaError_t launch_rmsnorm_t(const T* x, const T* z, const float* w, floa
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int tpr = dim / 8;
   const int64_t rpb = 256 / tpr;
-  int64_t blocks = (rows + rpb - 1) / rpb;
-  const int64_t cap = (int64_t)sms * 8;
-  if (blocks > cap) blocks = cap;
+  // enough blocks for one pass of RMS_U rows per thread, at most one wave of resident blocks
+  int64_t blocks = (rows + rpb * RMS_U - 1) / (rpb * RMS_U);
+  auto run = [&](auto kern) {
+    int per_sm = 0;
+    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, 256, 0);
+    const int64_t cap = (int64_t)sms * (per_sm > 0 ? per_sm : 1);
+    if (blocks > cap) blocks = cap;
+    if (blocks < 1) blocks = 1;
+    kern<<<(unsigned)blocks, 256, 0, s>>>(x, z, w, eps, rows, y);
+  };
   switch (tpr) {
 #define GDN_RMS_CASE(N) \
-  case N: rmsnorm_gated_kernel<T, N><<<(unsigned)blocks, 256, 0, s>>>(x, z, w, eps, rows, y); break;
+  case N: run(rmsnorm_gated_kernel<T, N>); break;
     GDN_RMS_CASE(1)
     GDN_RMS_CASE(2)
     GDN_RMS_CASE(4)
