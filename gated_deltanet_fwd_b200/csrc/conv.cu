@@ -12,11 +12,11 @@
 // read and written as 512-byte coalesced segments.
 //
 // Memory-level parallelism comes from a private per-thread ring in shared memory: each thread
-// keeps DEPTH-2 tokens of its own channels in flight with cp.async (16-byte, L1-bypassing), and
+// keeps DEPTH-NT tokens of its own channels in flight with cp.async (16-byte, L1-bypassing), and
 // waits only for the oldest ones.  Because a thread reads back only the slots it filled itself,
 // no block-wide synchronisation is needed.  The last K-1 inputs live in registers as a circular
 // window whose rotation is unrolled, so no register moves are spent on shifting it, and tokens
-// are computed two at a time in packed fp32 (two lanes per instruction) so that the latency
+// are computed two or three at a time in packed fp32 (two lanes per instruction) so that the latency
 // chains of conv -> SiLU -> norm overlap.  The grid
 // is one wave (two blocks per SM for K <= 4), each block taking an equal share of the tokens of one
 // 2048-channel slab.  The L2 norm of a head is a shuffle reduction over the group's group/8
@@ -120,9 +120,12 @@ __global__ void __launch_bounds__(CONV_THREADS, conv_blocks_per_sm(K)) conv_silu
   constexpr int DEPTH = CONV_RING_BYTES / (16 * V);  // ring slots per thread
   constexpr uint32_t SLOT = V * CONV_THREADS * 16;   // bytes per ring slot (whole block)
   constexpr int W = K > 1 ? K - 1 : 1;               // window length
-  // tokens per unrolled group: a multiple of W (the window returns to phase 0) and of 2 (tokens
-  // go in pairs)
-  constexpr int U = W >= 4 ? (W % 2 ? 2 * W : W) : W * (8 / W);
+  // tokens computed side by side: three where the window length allows a group of two triples
+  // (and the registers allow: bf16), else two
+  constexpr int NT = (W % 3 == 0 && sizeof(T) == 2) ? 3 : 2;
+  // tokens per unrolled group: a multiple of W (the window returns to phase 0) and of NT
+  constexpr int U = NT == 3 ? 6 : (W >= 4 ? (W % 2 ? 2 * W : W) : W * (8 / W));
+  static_assert(U % W == 0 && U % NT == 0, "group must hold whole windows and whole steps");
   static_assert((DEPTH & (DEPTH - 1)) == 0, "ring depth must be a power of two");
   extern __shared__ __align__(16) uint4 conv_ring[];
 
@@ -178,17 +181,18 @@ __global__ void __launch_bounds__(CONV_THREADS, conv_blocks_per_sm(K)) conv_silu
     }
     cp_async_commit();
   };
-  // Before token t_begin + i is taken, tokens up to i + DEPTH - 3 have been issued.  Taking
-  // NT (1 or 2) tokens refills the NT slots consumed by the previous step (their values are
-  // already in registers and used), then waits until token i + NT - 1 has landed: DEPTH - 2
-  // newer groups may still be in flight.
+  // Before token t_begin + i is taken, tokens up to i + DEPTH - NT - 1 have been issued.
+  // Taking m <= NT tokens refills m of the NT slots before token i, all consumed by earlier
+  // steps (their values are already in registers and used), then waits until token i + m - 1
+  // has landed: DEPTH - NT newer groups may still be in flight.
   auto take = [&](auto nt, int64_t i, float2 (*xt)[4]) {
-    constexpr int NT = decltype(nt)::value;
+    constexpr int M = decltype(nt)::value;
+    static_assert(M <= NT, "a step takes at most NT tokens");
 #pragma unroll
-    for (int k = 0; k < NT; ++k) issue(i + k + DEPTH - 2);
-    cp_async_wait<DEPTH - 2>();
+    for (int k = 0; k < M; ++k) issue(i + k + DEPTH - NT);
+    cp_async_wait<DEPTH - NT>();
 #pragma unroll
-    for (int k = 0; k < NT; ++k) {
+    for (int k = 0; k < M; ++k) {
       if (chan_ok) {
         ring_to_float2(ring + (uint32_t)((i + k) & (DEPTH - 1)) * SLOT, x, xt[k]);
       } else {
@@ -198,7 +202,7 @@ __global__ void __launch_bounds__(CONV_THREADS, conv_blocks_per_sm(K)) conv_silu
     }
   };
 #pragma unroll 1
-  for (int i = 0; i < DEPTH - 2; ++i) issue(i);
+  for (int i = 0; i < DEPTH - NT; ++i) issue(i);
 
   int n = seq_of_token(cu, N, Tlen, t_begin);
   int64_t s_beg, s_end;
@@ -234,15 +238,15 @@ __global__ void __launch_bounds__(CONV_THREADS, conv_blocks_per_sm(K)) conv_silu
     }
   };
 
-  // conv + SiLU + (optional) head L2 norm + store of NT consecutive tokens from t.  The window
-  // order is rotated by `ph` (token t's oldest input sits in win[ph]); each token overwrites its
-  // oldest slot with its own input, which the next token then sees as its newest.  Two tokens
-  // are computed side by side, so their dependency chains overlap.
+  // conv + SiLU + (optional) head L2 norm + store of M (NT or one) consecutive tokens from t.
+  // The window order is rotated by `ph` (token t's oldest input sits in win[ph]); each token
+  // overwrites its oldest slot with its own input, which the next token then sees as its newest.
+  // The tokens of a step are computed side by side, so their dependency chains overlap.
   auto tokens = [&](auto nt, int64_t t, const float2 (*xt)[4], int ph) {
-    constexpr int NT = decltype(nt)::value;
-    float2 acc[NT][4];
+    constexpr int M = decltype(nt)::value;
+    float2 acc[M][4];
 #pragma unroll
-    for (int k = 0; k < NT; ++k) {
+    for (int k = 0; k < M; ++k) {
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
         float2 a = bs[q];
@@ -256,13 +260,13 @@ __global__ void __launch_bounds__(CONV_THREADS, conv_blocks_per_sm(K)) conv_silu
       }
     }
 #pragma unroll
-    for (int k = 0; k < NT; ++k)
+    for (int k = 0; k < M; ++k)
 #pragma unroll
       for (int q = 0; q < 4; ++q) acc[k][q] = silu2(acc[k][q]);
     if (warp_norm) {
-      float ss[NT];
+      float ss[M];
 #pragma unroll
-      for (int k = 0; k < NT; ++k) {
+      for (int k = 0; k < M; ++k) {
         float2 s2 = __fmul2_rn(acc[k][0], acc[k][0]);
 #pragma unroll
         for (int q = 1; q < 4; ++q) s2 = __ffma2_rn(acc[k][q], acc[k][q], s2);
@@ -272,10 +276,10 @@ __global__ void __launch_bounds__(CONV_THREADS, conv_blocks_per_sm(K)) conv_silu
       for (int o = 16; o > 0; o >>= 1)
         if (o < lanes_per_group) {
 #pragma unroll
-          for (int k = 0; k < NT; ++k) ss[k] += __shfl_xor_sync(0xffffffffu, ss[k], o);
+          for (int k = 0; k < M; ++k) ss[k] += __shfl_xor_sync(0xffffffffu, ss[k], o);
         }
 #pragma unroll
-      for (int k = 0; k < NT; ++k) {
+      for (int k = 0; k < M; ++k) {
         const float inv = do_norm ? rsqrtf(ss[k] + l2_eps) : 1.0f;
 #pragma unroll
         for (int q = 0; q < 4; ++q) acc[k][q] = __fmul2_rn(acc[k][q], make_float2(inv, inv));
@@ -283,11 +287,11 @@ __global__ void __launch_bounds__(CONV_THREADS, conv_blocks_per_sm(K)) conv_silu
     }
     if (chan_ok) {
 #pragma unroll
-      for (int k = 0; k < NT; ++k) store8x2(y + (t + k) * C + c0, acc[k]);
+      for (int k = 0; k < M; ++k) store8x2(y + (t + k) * C + c0, acc[k]);
     }
   };
   using One = std::integral_constant<int, 1>;
-  using Two = std::integral_constant<int, 2>;
+  using Step = std::integral_constant<int, NT>;
 
   int64_t t = t_begin;
   if (t >= s_beg && t < s_end) fill_window(t);
@@ -314,10 +318,10 @@ __global__ void __launch_bounds__(CONV_THREADS, conv_blocks_per_sm(K)) conv_silu
     // groups of U tokens: the window rotates through all W phases and returns to phase 0
     while (t + U <= seg_end) {
 #pragma unroll
-      for (int u = 0; u < U; u += 2) {
-        float2 xt[2][4];
-        take(Two{}, t + u - t_begin, xt);
-        tokens(Two{}, t + u, xt, u % W);
+      for (int u = 0; u < U; u += NT) {
+        float2 xt[NT][4];
+        take(Step{}, t + u - t_begin, xt);
+        tokens(Step{}, t + u, xt, u % W);
       }
       t += U;
     }
