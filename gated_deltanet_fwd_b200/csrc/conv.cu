@@ -16,8 +16,8 @@
 // waits only for the oldest ones.  Because a thread reads back only the slots it filled itself,
 // no block-wide synchronisation is needed.  The last K-1 inputs live in registers as a circular
 // window whose rotation is unrolled, so no register moves are spent on shifting it, and tokens
-// are computed two or three at a time in packed fp32 (two lanes per instruction) so that the latency
-// chains of conv -> SiLU -> norm overlap.  The grid
+// are computed two or three at a time in packed fp32 (two lanes per instruction) so that the
+// latency chains of conv -> SiLU -> norm overlap.  The grid
 // is one wave (two blocks per SM for K <= 4), each block taking an equal share of the tokens of one
 // 2048-channel slab.  The L2 norm of a head is a shuffle reduction over the group's group/8
 // lanes, skipped by warps that hold only v channels.
@@ -357,10 +357,10 @@ __global__ void __launch_bounds__(CONV_THREADS, conv_blocks_per_sm(K)) conv_silu
 }
 
 template <typename T, int K>
-static cudaError_t launch_conv_k(int sms, int64_t n_tok, int slabs, const T* x, const float* w, const float* bias,
-                                 int64_t T_, int C, const int32_t* cu, int N, int n_l2, int group,
-                                 float l2_eps, const float* cs_in, float* cs_out, T* y,
-                                 cudaStream_t s) {
+static cudaError_t launch_conv_k(int sms, int64_t n_tok, int slabs, const T* x, const float* w,
+                                 const float* bias, int64_t T_, int C, const int32_t* cu, int N,
+                                 int n_l2, int group, float l2_eps, const float* cs_in,
+                                 float* cs_out, T* y, cudaStream_t s) {
   // one wave: every resident block slot gets an equal share of one slab's tokens
   int64_t cols = ((int64_t)sms * conv_blocks_per_sm(K) + slabs - 1) / slabs;
   const int64_t by_len = (n_tok + CONV_MIN_TOKENS - 1) / CONV_MIN_TOKENS;
