@@ -47,11 +47,11 @@ CHUNK_FLOP_PER_TOKEN_HEAD = 8 * 64 * 128 + 6 * 128 * 128
 # capture each (summaries under profiles/), tied to the kernel source they were taken from: once
 # the source changes the bench reports traffic as null until it is captured again.
 MEASURED_TRAFFIC = {
-    # chunk_tc_kernel on B=1, T=4096 (prefill 4K): 68.2 MB read + 7.4 MB written = 18,455 B per
+    # chunk_tc_kernel on B=1, T=4096 (prefill 4K): 68.2 MB read + 8.8 MB written = 18,805 B per
     # token over all 32 heads; scaled by the tokens of a launch (reads scale with tokens; the
     # write count is a lower bound, the output drains from L2 after the kernel).
-    "gdn_chunk_fwd": dict(source="csrc/chunk_tc.cu", sha256_16="9357e5e1e408224c",
-                          bytes_per_token=75590144 / 4096),
+    "gdn_chunk_fwd": dict(source="csrc/chunk_tc.cu", sha256_16="d91b1956d8eb683c",
+                          bytes_per_token=77027072 / 4096),
     # recurrent_step_kernel on 256 sequences x 32 heads: 5.92 TB/s x 172.8 us.
     "gdn_recurrent_step": dict(source="csrc/recurrent.cu", sha256_16="b07ec22be73c2392",
                                bytes_per_launch=1.0224e9),
