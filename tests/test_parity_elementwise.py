@@ -75,6 +75,36 @@ def test_conv_varlen_with_state(dtype):
     assert max_abs(s_out, s_ref) == 0.0
 
 
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+@pytest.mark.parametrize("K", [2, 5, 6, 7])
+def test_conv_ragged_slabs_and_groups(dtype, K):
+    """Channel count that leaves a partial warp in a second channel slab (2056 = 2048 + 8),
+    32-channel norm groups whose normalised range ends inside a warp (1184 channels), window
+    lengths on every unrolling path, and ragged varlen sequences (empty, shorter than K-1, long
+    enough to split across blocks) with a carried state."""
+    gen = torch.Generator().manual_seed(40 + K)
+    C, n_l2, group = 2056, 1184, 32
+    cu = [0, 3, 3, 200, 201, 777, 1000]
+    N, T = len(cu) - 1, cu[-1]
+    x = torch.randn(1, T, C, generator=gen).to(inputs.torch_dtype(dtype))
+    w = (torch.rand(C, K, generator=gen) * 2 - 1) / K ** 0.5
+    bias = torch.randn(C, generator=gen) * 0.1
+    s_in = torch.randn(N, C, K - 1, generator=gen)
+    cu_t = torch.tensor(cu, dtype=torch.int32)
+    s_out = torch.empty(N, C, K - 1, device=DEV)
+    y = gdn.gdn_causal_conv1d_silu(x.to(DEV), w.to(DEV), bias.to(DEV), cu_seqlens=cu_t.to(DEV),
+                                   n_l2norm_ch=n_l2, l2norm_group=group,
+                                   conv_state_in=s_in.to(DEV), conv_state_out=s_out)
+    ref, s_ref = oracle.causal_conv1d_silu(x, w, bias, cu_seqlens=cu_t, n_l2norm_ch=n_l2,
+                                           l2norm_group=group, conv_state_in=s_in,
+                                           return_state=True)
+    if dtype == "bf16":
+        assert_bf16_rounding_close(y, ref, "conv y")
+    else:
+        assert_f32_close(y, ref, "conv y", tol=1e-5)
+    assert max_abs(s_out, s_ref) == 0.0
+
+
 def test_conv_layer_core_full_size_sampled():
     """Layer-core size (B=2, T=16384, 8192 channels, K=4) in the launch the bench times; the
     oracle checks a channel subset (the conv is depthwise, the L2 norm per whole head)."""
