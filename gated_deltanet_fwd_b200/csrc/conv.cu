@@ -17,10 +17,10 @@
 // no block-wide synchronisation is needed.  The last K-1 inputs live in registers as a circular
 // window whose rotation is unrolled, so no register moves are spent on shifting it, and tokens
 // are computed two or three at a time in packed fp32 (two lanes per instruction) so that the
-// latency chains of conv -> SiLU -> norm overlap.  The grid
-// is one wave (two blocks per SM for K <= 4), each block taking an equal share of the tokens of one
-// 2048-channel slab.  The L2 norm of a head is a shuffle reduction over the group's group/8
-// lanes, skipped by warps that hold only v channels.
+// latency chains of conv -> SiLU -> norm overlap.  The grid is one wave (two blocks per SM for
+// K <= 4), each block taking an equal share of the tokens of one 2048-channel slab.  The L2 norm
+// of a head is a shuffle reduction over the group's group/8 lanes, skipped by warps that hold
+// only v channels.
 #include <type_traits>
 
 #include "gdn_internal.cuh"
