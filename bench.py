@@ -456,6 +456,54 @@ def run_reference(args, dist):
     return 0
 
 
+# ------------------------------------------------------------------ profiling -------------
+
+def run_profile(mode, reps):
+    """Runs one workload a few times and nothing else, for ncu captures (few launches, at most a
+    few GB on the device):
+
+    prefill    gdn_gates + gdn_chunk_fwd on the 32768-token varlen workload (4 sequences)
+    prefill4k  gdn_gates + gdn_chunk_fwd on B=1, T=4096
+    decode     consecutive gdn_gates + gdn_recurrent_step calls on 256 sequences x 32 heads
+    conv       gdn_causal_conv1d_silu on the [2, 16384, 8192] mix, then gdn_gated_rmsnorm on the
+               v channels viewed as 128-wide rows
+    """
+    from gated_deltanet_fwd_b200 import gdn
+    dev = torch.device("cuda", 0)
+    if mode in ("prefill", "prefill4k"):
+        name = "prefill_varlen_32k" if mode == "prefill" else "prefill_4k"
+        w = inputs.WORKLOADS[name]
+        x = inputs.rule_inputs(**w, seed=1000 + w["index"])
+        d = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in x.items()}
+        for _ in range(reps):
+            g, beta = gdn.gdn_gates(d["a"], d["b"], d["A_log"], d["dt_bias"])
+            gdn.gdn_chunk_fwd(d["q"], d["k"], d["v"], g, beta, initial_state=d["initial_state"],
+                              cu_seqlens=d["cu_seqlens"], chunk=w["chunk"])
+    elif mode == "decode":
+        w = dict(inputs.WORKLOADS["decode_256"], steps=max(reps, 1))
+        x = inputs.decode_inputs(**w, seed=1000 + w["index"])
+        st = x["state"].to(dev)
+        A_log, dt_bias = x["A_log"].to(dev), x["dt_bias"].to(dev)
+        for s in range(w["steps"]):
+            g, beta = gdn.gdn_gates(x["a"][s].to(dev), x["b"][s].to(dev), A_log, dt_bias)
+            gdn.gdn_recurrent_step(x["q"][s].to(dev), x["k"][s].to(dev), x["v"][s].to(dev), g,
+                                   beta, st)
+    elif mode == "conv":
+        w = inputs.WORKLOADS["layer_core_2x16k"]
+        x = inputs.layer_core_inputs(**w, seed=1000 + w["index"])
+        mix, cw = x["mix"].to(dev), x["conv_w"].to(dev)
+        z, nw = x["z"].to(dev).view(-1, w["dv"]), x["norm_w"].to(dev)
+        nqk = 2 * w["Hk"] * w["dk"]
+        for _ in range(reps):
+            y = gdn.gdn_causal_conv1d_silu(mix, cw, None, n_l2norm_ch=nqk, l2norm_group=w["dk"])
+            gdn.gdn_gated_rmsnorm(y[:, :, nqk:].contiguous().view(-1, w["dv"]), z, nw)
+    else:
+        raise SystemExit(run_profile.__doc__)
+    torch.cuda.synchronize()
+    print("done", mode, flush=True)
+    return 0
+
+
 # ------------------------------------------------------------------ main -------------------
 
 def main():
@@ -465,7 +513,12 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--profile", default=None,
+                    help="run one workload for a profiler capture: prefill|prefill4k|decode|conv")
+    ap.add_argument("--repeats", type=int, default=2, help="launches per --profile run")
     args = ap.parse_args()
+    if args.profile:
+        return run_profile(args.profile, args.repeats)
     args.warmup = max(args.warmup, 3)
     dist = Dist()
     if args.impl == "reference":
@@ -480,8 +533,12 @@ def main():
     clocks.start()
     pre = bench_prefill(dist, gdn, args.steps, args.warmup, peaks)
     clk = clocks.stop()
+    clocks.start()
     dec = bench_decode(dist, gdn, max(2, args.steps // 4), args.warmup, peaks)
+    dec["clocks"] = clocks.stop()
+    clocks.start()
     core = bench_layer_core(dist, gdn, max(2, args.steps // 4), args.warmup, peaks)
+    core["clocks"] = clocks.stop()
     cpu = None
     if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline:
         r, cores, desc = oracle_prefill_sample()

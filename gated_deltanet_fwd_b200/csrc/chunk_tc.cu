@@ -241,6 +241,9 @@ __global__ void __launch_bounds__(TC_THREADS, 1) chunk_tc_kernel(
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + OFF_BAR + N_BARS * 8);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + OFF_BAR + N_BARS * 8 + 4);
+  // prep CTA: number of [T'; P] bulk copies its leader has issued into the chain CTA (read by the
+  // chain CTA at exit, so that no copy can still be landing in its shared memory when it leaves)
+  volatile int* prep_issued = reinterpret_cast<volatile int*>(smem + OFF_BAR + N_BARS * 8 + 8);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const uint32_t rank = cluster_rank();  // 0 = prep, 1 = chain
@@ -277,6 +280,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) chunk_tc_kernel(
     mbar_init(&bars[B_M_S], 1);
     mbar_init(&bars[B_DRAIN], 1);
     *abort_flag = 0;
+    *prep_issued = 0;
     fence_barrier_init();
     // the chain CTA expects one [T'; P] tile per chunk from the prep CTA's bulk copies
     if (rank == 1) {
@@ -297,6 +301,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) chunk_tc_kernel(
     report(P.status, code);
     *abort_flag = 1;
   };
+  int tp_consumed_final = 0;  // chain leader: [T'; P] arrivals it waited for
 
   if (warp == PRODUCER_WARP) {
     // ------------------------------------------------------------ TMA producers -----------
@@ -564,16 +569,19 @@ __global__ void __launch_bounds__(TC_THREADS, 1) chunk_tc_kernel(
       named_bar(1, TC_WORKERS);
       TC_TS(12);
       // the chain CTA arms its barrier for these bytes itself; the copy only completes them
-      if (leader)
+      if (leader) {
         bulk_copy_to_peer(peer_addr(sbase + CH_TP + b * TP_BUF, 1), smem_u32(tpl), TP_BUF,
                           peer_addr(smem_u32(&bars[B_PREP_FULL0 + b]), 1));
+        *prep_issued = c + 1;
+      }
       TC_TS(6);
     }
     TC_TRACE_FLUSH(2);
     if (warp == 0) cp_async_wait_all();  // no gate copy may still be landing at exit
     if (leader) {
+      // every D1 MMA has completed before the CTA releases its tensor memory
       mma_commit(&bars[B_DRAIN]);
-      mbar_wait(&bars[B_DRAIN], 0);
+      if (!mbar_wait(&bars[B_DRAIN], 0)) report(P.status, GDN_ERR_TIMEOUT);
     }
   } else {
     // ------------------------------------------------------------ chain CTA (512 threads) --
@@ -659,6 +667,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) chunk_tc_kernel(
     };
     float g_row_prev = 0.0f;
     bool all_ok = true;
+    int tp_consumed = 0;  // [T'; P] copies whose arrival the leader has waited for
 
     // Exits are decided jointly (named_bar_and): a wait that ran out in any thread makes all 512
     // leave at the same barrier.
@@ -750,6 +759,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) chunk_tc_kernel(
       TC_TS(2);
       // step 3: D_U = [T'; P] X  (needs this chunk's T' and P from the prep CTA)
       ok = !leader || mbar_wait(&bars[B_PREP_FULL0 + b], (c >> 1) & 1);
+      if (leader && ok) tp_consumed = c + 1;
       // re-arm the buffer's barrier for chunk c + 2, whose copy the prep CTA can only start
       // after this chunk hands the buffer back
       if (leader && ok && c + 2 < nchunks) mbar_arrive_expect_tx(&bars[B_PREP_FULL0 + b], TP_BUF);
@@ -840,9 +850,13 @@ __global__ void __launch_bounds__(TC_THREADS, 1) chunk_tc_kernel(
     TC_TRACE_FLUSH(leader ? 3 : 4);
     if (warp == 0) cp_async_wait_all();  // no gate copy may still be landing at exit
     if (leader) {
+      // after an abort MMAs may still be in flight: wait for all of them before tensor memory
+      // is read or released; if even that wait runs out, the state is not read back
       mma_commit(&bars[B_DRAIN]);
-      mbar_wait(&bars[B_DRAIN], 0);
+      if (!mbar_wait(&bars[B_DRAIN], 0)) fail(GDN_ERR_TIMEOUT);
     }
+    named_bar(1, TC_WORKERS);  // the leader's drain result is visible to every worker
+    tp_consumed_final = tp_consumed;
     if (P.S_T && !*abort_flag) {
       float sv[32];
       tmem_ld32(s_tm, sv);
@@ -851,8 +865,24 @@ __global__ void __launch_bounds__(TC_THREADS, 1) chunk_tc_kernel(
     }
   }
 
-  // neither CTA leaves while the other may still touch its shared memory
+  // Neither CTA leaves while the other may still touch its shared memory.  After this barrier the
+  // prep CTA issues nothing more; a [T'; P] copy it issued that the chain CTA never waited for
+  // (only after an abort) may still be landing in the chain CTA, so the chain leader waits for
+  // those arrivals (bounded) before the final barrier lets both CTAs go.
   tc_fence_before();
+  cluster_sync();
+  if (rank == 1 && tid == 0) {
+    uint32_t issued_remote;
+    asm volatile("ld.shared::cluster.u32 %0, [%1];"
+                 : "=r"(issued_remote)
+                 : "r"(peer_addr(smem_u32((const void*)prep_issued), 0))
+                 : "memory");
+    for (int c = tp_consumed_final; c < (int)issued_remote; ++c)
+      if (!mbar_wait(&bars[B_PREP_FULL0 + (c & 1)], (uint32_t)(c >> 1) & 1)) {
+        report(P.status, GDN_ERR_TIMEOUT);
+        break;
+      }
+  }
   cluster_sync();
   if (warp == 0) {
     tc_fence_after();

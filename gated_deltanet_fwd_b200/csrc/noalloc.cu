@@ -9,36 +9,24 @@
 //
 // The array is a file-scope __device__ variable: every GPU that loads the library holds it until
 // the process exits.  In host code its name is only a host-side stand-in, not a device address,
-// so the device address is looked up with cudaGetSymbolAddress once per device (with that device
-// current) and cached; that lookup happens on the first call on each device.
-#include <mutex>
-
+// so every call looks up the array's device address on the current device with
+// cudaGetSymbolAddress (a lookup that allocates nothing).  Looking it up on every call rather
+// than caching it keeps the address right after a cudaDeviceReset, which reloads the module.
 #include "gdn_internal.cuh"
 
 namespace {
 
-constexpr size_t kNoAllocScratchBytes = 64 * 1024;  // GDN_NOALLOC_SCRATCH_BYTES in gdn.h
-constexpr int kMaxDevices = 64;
+constexpr size_t kNoAllocScratchBytes = GDN_NOALLOC_SCRATCH_BYTES;
+static_assert(kNoAllocScratchBytes % 256 == 0, "scratch keeps the workspace alignment");
 
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 
-std::mutex g_scratch_mutex;
-void* g_scratch_addr[kMaxDevices] = {};
-
-// Device address of g_noalloc_scratch on the current device, looked up once per device.
+// Device address of g_noalloc_scratch on the current device.
 cudaError_t scratch_address(void** out) {
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
+  void* p = nullptr;
+  cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
   if (e != cudaSuccess) return e;
-  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
-  std::lock_guard<std::mutex> lock(g_scratch_mutex);
-  if (!g_scratch_addr[dev]) {
-    void* p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
-    if (e != cudaSuccess) return e;
-    g_scratch_addr[dev] = p;
-  }
-  *out = g_scratch_addr[dev];
+  *out = p;
   return cudaSuccess;
 }
 

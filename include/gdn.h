@@ -156,8 +156,9 @@ gdn_status gdn_chunk_fwd_strided(const void* q, int64_t q_tok_stride, const void
  * variable that every GPU which loads the library holds until the process exits).  Sizes whose
  * gdn_chunk_fwd_workspace_size() exceeds that maximum return GDN_ERR_UNSUPPORTED.  The call
  * allocates nothing (no cudaMalloc, cudaFree or allocating library routine).
- * The first call on each device looks up the array's device address (cudaGetSymbolAddress) with
- * that device current; make that first call before any stream capture.  All calls on a device
+ * Every call looks up the array's device address (cudaGetSymbolAddress) on the current device; the
+ * first call on a device may load the library's device code there, so make that first call
+ * before any stream capture.  cudaDeviceReset between calls is fine.  All calls on a device
  * share the one array and it keeps the last call's contents (the status word is cleared by each
  * call), so calls whose kernels overlap on the GPU -- on different streams, or from different host
  * threads -- race on it: serialise them.  Device-detected faults land in that shared status word

@@ -1,5 +1,8 @@
 """Shared helpers of the GPU parity tests: error metrics, tolerances, and per-(sequence, head)
 oracle sampling for full-size workloads.  No arithmetic of the method lives here."""
+import json
+import os
+
 import numpy as np
 import torch
 
@@ -29,14 +32,27 @@ def max_abs(x, ref):
     return float(np.max(np.abs(x - ref))) if x.size else 0.0
 
 
+def record_margin(what, **metrics):
+    """Prints the measured error next to its tolerance (shown with `pytest -s` or `-rA`) and,
+    when GDN_MARGINS names a file, appends it there as one JSON line."""
+    print("MARGIN " + what + " " + " ".join(f"{k}={v:.3e}" if isinstance(v, float) else f"{k}={v}"
+                                            for k, v in metrics.items()), flush=True)
+    path = os.environ.get("GDN_MARGINS")
+    if path:
+        with open(path, "a") as f:
+            f.write(json.dumps(dict(what=what, **metrics)) + "\n")
+
+
 def assert_bf16_close(x, ref, what=""):
     r, m = rel_l2(x, ref), max_abs(x, ref)
+    record_margin(what, rel_l2=r, rel_l2_tol=BF16_REL_L2, max_abs=m, max_abs_tol=BF16_MAX_ABS)
     assert r <= BF16_REL_L2 and m <= BF16_MAX_ABS, f"{what}: rel_L2={r:.3e} max_abs={m:.3e}"
     return r, m
 
 
 def assert_f32_close(x, ref, what="", tol=F32_REL):
     r = rel_l2(x, ref)
+    record_margin(what, rel_l2=r, rel_l2_tol=tol)
     assert r <= tol, f"{what}: rel_L2={r:.3e} > {tol:.1e}"
     return r
 
@@ -53,6 +69,8 @@ def assert_bf16_rounding_close(x, ref, what="", abs_floor=1e-6):
     err = np.abs(x - ref)
     bound = (BF16_UNIT_ROUNDOFF + 1e-5) * np.abs(ref) + abs_floor
     bad = err > bound
+    record_margin(what, worst_err_over_bound=float(np.max(err / bound)) if err.size else 0.0,
+                  rel_l2=rel_l2(x, ref))
     assert not bad.any(), (f"{what}: {int(bad.sum())} elements beyond bf16 rounding, worst "
                            f"err {err[bad].max():.3e} at |ref| {np.abs(ref[bad]).max():.3e}")
     return rel_l2(x, ref)

@@ -1,17 +1,17 @@
 """GPU parity of gdn_chunk_fwd (chunked prefill) against the fp64 oracle.
 
-Small cases are compared element by element on every output; the full-size workloads run in the
-launch configuration the bench times and are compared on sampled (sequence, v-head) units, each of
-which the oracle can compute on its own.
+Every case, the full-size workloads included, is compared element by element on every output
+and every final state; the full-size workloads run in the launch configuration the bench times.
 """
+import os
+
 import numpy as np
 import pytest
 import torch
 
 import oracle
 from gated_deltanet_fwd_b200 import gdn, inputs
-from gdn_testutil import (assert_bf16_close, assert_f32_close, oracle_gates_f32, oracle_units,
-                          rel_l2)
+from gdn_testutil import assert_bf16_close, assert_f32_close, oracle_gates_f32
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -28,10 +28,13 @@ def _gpu_chunk(x, g, beta, chunk, scale):
     return out.cpu(), S.cpu()
 
 
+NTHREADS = max(1, os.cpu_count() or 1)
+
+
 def _full_oracle(x, g, beta, scale):
     return oracle.gated_delta_rule(x["q"], x["k"], x["v"], g, beta, scale,
                                    initial_state=x["initial_state"],
-                                   cu_seqlens=x["cu_seqlens"], nthreads=8)
+                                   cu_seqlens=x["cu_seqlens"], nthreads=NTHREADS)
 
 
 def _check(dtype, out, S, o_ref, S_ref, what):
@@ -101,40 +104,49 @@ def test_chunk_empty_and_no_state():
     _check("bf16", out, S, o_ref, S_ref, "no S0")
 
 
-def _sampled(wname, units, a_mean=0.0):
+def _full_size(wname, a_mean=0.0):
+    """A full-size workload on the GPU against the oracle over every element of `out` and every
+    final state."""
     w = inputs.WORKLOADS[wname]
     x = inputs.rule_inputs(**w, seed=1000 + w["index"], a_mean=a_mean)
     g, beta = oracle_gates_f32(x)
     scale = w["dk"] ** -0.5
     out, S = _gpu_chunk(x, g, beta, w["chunk"], scale)
-    ref = oracle_units(x["q"], x["k"], x["v"], g, beta, scale, x["initial_state"],
-                       x["cu_seqlens"], units)
-    cu = x["cu_seqlens"]
-    for (n, h), (o_ref, S_ref) in ref.items():
-        if cu is not None:
-            o = out[0, int(cu[n]):int(cu[n + 1]), h]
-        else:
-            o = out[n, :, h]
-        assert_bf16_close(o, o_ref, f"{wname} unit {(n, h)} out")
-        assert_bf16_close(S[n, h], S_ref, f"{wname} unit {(n, h)} state")
+    o_ref, S_ref = _full_oracle(x, g, beta, scale)
+    tag = f"{wname} a_mean={a_mean}"
+    assert_bf16_close(out, o_ref, tag + " out (all elements)")
+    assert_bf16_close(S, S_ref, tag + " final states (all)")
 
 
-def test_prefill_4k_sampled():
+def test_prefill_4k_full():
     """B=1, T=4096, 16 q/k heads, 32 v heads, d=128, bf16, chunk 64, zero initial state."""
-    _sampled("prefill_4k", [(0, 0), (0, 1), (0, 17), (0, 31)])
+    _full_size("prefill_4k")
 
 
-def test_prefill_4k_slow_decay_sampled():
-    _sampled("prefill_4k", [(0, 3), (0, 30)], a_mean=-6.0)
+def test_prefill_4k_slow_decay_full():
+    _full_size("prefill_4k", a_mean=-6.0)
 
 
-def test_prefill_varlen_32k_sampled():
+def test_prefill_varlen_32k_full():
     """32768 tokens as 4 sequences (16384/8192/6144/2048) with per-sequence initial states."""
-    _sampled("prefill_varlen_32k", [(0, 0), (1, 9), (2, 20), (3, 31)])
+    _full_size("prefill_varlen_32k")
 
 
-def test_prefill_varlen_32k_slow_decay_sampled():
-    _sampled("prefill_varlen_32k", [(0, 5), (3, 16)], a_mean=-6.0)
+def test_prefill_varlen_32k_slow_decay_full():
+    _full_size("prefill_varlen_32k", a_mean=-6.0)
+
+
+def test_prefill_16k_zero_decay_long_chain():
+    """One 16384-token sequence with g = 0: nothing forgets, so any rounding the chunk path
+    carries from chunk to chunk (its state operand is rounded to bf16 every chunk) accumulates
+    over all 256 chunks instead of being damped away."""
+    x = inputs.rule_inputs(B=1, T=16384, Hk=1, Hv=2, dk=128, dv=128, seed=16384, s0_std=0.02)
+    g, beta = oracle_gates_f32(x)
+    g = torch.zeros_like(g)
+    out, S = _gpu_chunk(x, g, beta, 64, 128 ** -0.5)
+    o_ref, S_ref = _full_oracle(x, g, beta, 128 ** -0.5)
+    assert_bf16_close(out, o_ref, "16k g=0 out")
+    assert_bf16_close(S, S_ref, "16k g=0 final state")
 
 
 @pytest.mark.parametrize("chunk,dtype", [(64, "bf16"), (32, "bf16"), (16, "f32")])

@@ -105,22 +105,6 @@ def test_conv_ragged_slabs_and_groups(dtype, K):
     assert max_abs(s_out, s_ref) == 0.0
 
 
-def test_conv_layer_core_full_size_sampled():
-    """Layer-core size (B=2, T=16384, 8192 channels, K=4) in the launch the bench times; the
-    oracle checks a channel subset (the conv is depthwise, the L2 norm per whole head)."""
-    w_ = inputs.WORKLOADS["layer_core_2x16k"]
-    x = inputs.layer_core_inputs(**w_, seed=1000 + w_["index"])
-    Hk, Hv, d = w_["Hk"], w_["Hv"], w_["dk"]
-    y = gdn.gdn_causal_conv1d_silu(x["mix"].to(DEV), x["conv_w"].to(DEV), None,
-                                   n_l2norm_ch=2 * Hk * d, l2norm_group=d).cpu()
-    heads = [0, 5, Hk + 3, 2 * Hk + 0, 2 * Hk + 31]  # two q heads, one k head, two v heads
-    ch = torch.cat([torch.arange(h * d, (h + 1) * d) for h in heads])
-    n_norm = 3 * d  # the first three selected groups are q/k heads
-    ref = oracle.causal_conv1d_silu(x["mix"][:, :, ch], x["conv_w"][ch], None,
-                                    n_l2norm_ch=n_norm, l2norm_group=d)
-    assert_bf16_rounding_close(y[:, :, ch], ref, "conv y (sampled channels)")
-
-
 @pytest.mark.parametrize("dtype", ["bf16", "f32"])
 @pytest.mark.parametrize("dim", [64, 128, 256])
 def test_gated_rmsnorm(dtype, dim):
@@ -146,6 +130,5 @@ def test_gated_rmsnorm_in_place_layer_core_size():
     w = torch.randn(128, generator=gen) * 0.02
     xd = x.to(DEV)
     y = gdn.gdn_gated_rmsnorm(xd, z.to(DEV), w.to(DEV), eps=1e-6, y=xd)  # in place
-    idx = torch.randint(0, rows, (4096,), generator=gen)
-    ref = oracle.gated_rmsnorm(x[idx], z[idx], w, eps=1e-6)
-    assert_bf16_rounding_close(y.cpu()[idx], ref, "rmsnorm (sampled rows)")
+    ref = oracle.gated_rmsnorm(x, z, w, eps=1e-6)
+    assert_bf16_rounding_close(y.cpu(), ref, "rmsnorm in place, all rows")
