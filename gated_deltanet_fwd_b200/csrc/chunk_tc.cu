@@ -892,39 +892,6 @@ __global__ void __launch_bounds__(TC_THREADS, 1) chunk_tc_kernel(
 
 // ---------------------------------------------------------------- host side ---------------
 
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
-                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
-                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn() {
-  static EncodeTiledFn fn = nullptr;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
-            cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(p);
-  });
-  return fn;
-}
-
-// [rows, heads, 128] bf16 with `tok_stride` elements between rows -> 3D map {128, heads, rows},
-// box {64, 1, 64}, 128-byte swizzle.
-bool make_map(CUtensorMap* m, const void* base, int heads, int64_t rows, int64_t tok_stride) {
-  EncodeTiledFn enc = encode_fn();
-  if (!enc) return false;
-  cuuint64_t dims[3] = {128, (cuuint64_t)heads, (cuuint64_t)rows};
-  cuuint64_t strides[2] = {128 * 2, (cuuint64_t)tok_stride * 2};
-  cuuint32_t box[3] = {64, 1, 64};
-  cuuint32_t es[3] = {1, 1, 1};
-  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
-             es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 cudaError_t launch_chunk_tc_impl(const void* q, const void* k, const void* v, TokStrides ts,
                                  const float* g, const float* beta, float scale, const float* S0,
                                  const int32_t* cu, int N, int B, int64_t T, int Hk, int Hv,
@@ -936,8 +903,8 @@ cudaError_t launch_chunk_tc_impl(const void* q, const void* k, const void* v, To
   if (2 * units > 0x7fffffff) return cudaErrorInvalidConfiguration;
   CUtensorMap mq, mk, mv;
   const int64_t map_rows = rows > 0 ? rows : 1;
-  if (!make_map(&mq, q, Hk, map_rows, ts.q) || !make_map(&mk, k, Hk, map_rows, ts.k) ||
-      !make_map(&mv, v, Hv, map_rows, ts.v))
+  if (!make_tok_map(&mq, q, Hk, map_rows, ts.q) || !make_tok_map(&mk, k, Hk, map_rows, ts.k) ||
+      !make_tok_map(&mv, v, Hv, map_rows, ts.v))
     return cudaErrorInvalidValue;
   TcParams p;
   p.g = g;

@@ -5,6 +5,7 @@
 // and never trap.
 #include <stdio.h>
 
+#include "chunk_tm.cuh"
 #include "gdn_internal.cuh"
 
 using namespace gdn;
@@ -98,7 +99,9 @@ gdn_status gdn_causal_conv1d_silu(const void* x, gdn_dtype dtype, const float* w
 
 size_t gdn_chunk_fwd_workspace_size(int N, int B, int64_t T, int Hk, int Hv, int dk, int dv,
                                     int chunk) {
-  (void)N; (void)B; (void)T; (void)Hk; (void)Hv; (void)dk; (void)dv; (void)chunk;
+  (void)Hk;
+  if (dk == gdn::tm::D && dv == gdn::tm::D && chunk == gdn::tm::C && N >= 0 && B >= 0 && T >= 0 && Hv >= 1)
+    return (gdn::tm::workspace_bytes(N, (int64_t)B * T, Hv) + 255) & ~size_t(255);
   return kStatusBytes;
 }
 
@@ -132,8 +135,7 @@ gdn_status gdn_chunk_fwd_strided(const void* q, int64_t q_tok_stride, const void
       v_tok_stride < (int64_t)Hv * dv || q_tok_stride % 8 || k_tok_stride % 8 ||
       v_tok_stride % 8)
     return GDN_ERR_INVALID_ARG;
-  if (!workspace || workspace_bytes < gdn_chunk_fwd_workspace_size(N, B, T, Hk, Hv, dk, dv, chunk))
-    return GDN_ERR_INVALID_ARG;
+  if (!workspace || workspace_bytes < kStatusBytes) return GDN_ERR_INVALID_ARG;
   if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return GDN_ERR_INVALID_ARG;
   if (N == 0) return GDN_OK;
   const int64_t n_tok = (int64_t)B * T;
@@ -154,10 +156,18 @@ gdn_status gdn_chunk_fwd_strided(const void* q, int64_t q_tok_stride, const void
   if (cudaMemsetAsync(status, 0, sizeof(int), s) != cudaSuccess) return GDN_ERR_CUDA;
   const TokStrides ts{q_tok_stride, k_tok_stride, v_tok_stride};
   cudaError_t e;
-  if (dtype == GDN_BF16 && dk == 128 && dv == 128 && chunk == 64)
-    e = launch_chunk_tc(q, k, v, ts, g, beta, scale, initial_state, cu_seqlens, N, B, T, Hk, Hv,
-                        out, final_state, status, s);
-  else
+  if (dtype == GDN_BF16 && dk == gdn::tm::D && dv == gdn::tm::D && chunk == gdn::tm::C) {
+    if (workspace_bytes >= gdn::tm::workspace_bytes(N, (int64_t)B * T, Hv)) {
+      // prep kernel over all (chunk, k-head), then the chain over (sequence, v-head)
+      e = launch_chunk_prep(q, k, ts, g, beta, cu_seqlens, N, B, T, Hk, Hv, workspace, status, s);
+      if (e == cudaSuccess)
+        e = launch_chunk_chain(q, k, v, ts, scale, initial_state, cu_seqlens, N, B, T, Hk, Hv,
+                               out, final_state, workspace, status, s);
+    } else {
+      e = launch_chunk_tc(q, k, v, ts, g, beta, scale, initial_state, cu_seqlens, N, B, T, Hk,
+                          Hv, out, final_state, status, s);
+    }
+  } else
     e = launch_chunk_simt(q, k, v, ts, g, beta, dtype, scale, initial_state, cu_seqlens, N, B, T,
                           Hk, Hv, dk, dv, chunk, out, final_state, status, s);
   return from_cuda(e);

@@ -2,6 +2,7 @@
 // internal declarations.  Nothing here is exported.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -162,7 +163,24 @@ cudaError_t launch_chunk_simt(const void* q, const void* k, const void* v, TokSt
                               int dv, int chunk, void* out, float* S_T, int* status,
                               cudaStream_t s);
 
-// Tensor-core chunk path: bf16, dk = dv = 128, chunk = 64.
+// TMA tensor maps (tma_maps.cu), 128-byte swizzle, bf16:
+//   make_tok_map:    [rows, heads, 128] with `tok_stride` elements between rows; box {64, 1, 64}
+//   make_rows64_map: [rows, 64] dense;                                          box {64, box_rows}
+bool make_tok_map(CUtensorMap* m, const void* base, int heads, int64_t rows, int64_t tok_stride);
+bool make_rows64_map(CUtensorMap* m, const void* base, int64_t rows, uint32_t box_rows);
+
+// Two-kernel tensor-core prefill (bf16, dk = dv = 128, chunk = 64): the parallel prep kernel,
+// then the chain kernel.  `ws` holds at least tm::workspace_bytes(N, B*T, Hv) bytes.
+cudaError_t launch_chunk_prep(const void* q, const void* k, TokStrides ts, const float* g,
+                              const float* beta, const int32_t* cu, int N, int B, int64_t T,
+                              int Hk, int Hv, void* ws, int* status, cudaStream_t s);
+cudaError_t launch_chunk_chain(const void* q, const void* k, const void* v, TokStrides ts,
+                               float scale, const float* S0, const int32_t* cu, int N, int B,
+                               int64_t T, int Hk, int Hv, void* out, float* S_T, void* ws,
+                               int* status, cudaStream_t s);
+
+// Tensor-core chunk path without scratch (one CTA pair per sequence and head): bf16,
+// dk = dv = 128, chunk = 64.
 cudaError_t launch_chunk_tc(const void* q, const void* k, const void* v, TokStrides ts,
                             const float* g,
                             const float* beta, float scale, const float* S0, const int32_t* cu,

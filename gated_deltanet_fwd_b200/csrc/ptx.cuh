@@ -70,7 +70,13 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
 
 // Waits for the phase with the given parity to complete.  Gives up (returns false) after
 // kWaitLimitNs of wall-clock time or kSpinLimit polls, whichever comes first.
-constexpr uint64_t kWaitLimitNs = 4000000000ull;  // 4 s: every legitimate wait is microseconds
+// 4 s: every legitimate wait is microseconds.  The failure-test build of the library sets a
+// limit of about a millisecond (GDN_DEBUG_WAIT_NS) so that a test can make a wait run out quickly.
+#ifdef GDN_DEBUG_WAIT_NS
+constexpr uint64_t kWaitLimitNs = GDN_DEBUG_WAIT_NS;
+#else
+constexpr uint64_t kWaitLimitNs = 4000000000ull;
+#endif
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
@@ -177,6 +183,19 @@ __device__ __forceinline__ void mma_bf16_ss(uint32_t d_tmem, uint64_t a_desc, ui
       : "memory");
 }
 
+// D[tmem] (+)= A[tmem] x B[smem desc]^T, kind::f16: A is held in tensor memory (lane m = row m,
+// each 32-bit column two consecutive K elements, the lower K in the low half; a 16-deep K step
+// spans 8 columns), B comes from shared memory.
+__device__ __forceinline__ void mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                            uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 // Arrives on `bar` once every tcgen05.mma issued so far by this thread has completed.
 __device__ __forceinline__ void mma_commit(uint64_t* bar) {
   asm volatile(
@@ -225,6 +244,16 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const float (&v)[16]) 
       "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])), "r"(__float_as_uint(v[11])),
       "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])), "r"(__float_as_uint(v[14])),
       "r"(__float_as_uint(v[15]))
+      : "memory");
+}
+
+// 16 consecutive columns of raw 32-bit cells (e.g. packed bf16 pairs) into this warp's 32 lanes.
+__device__ __forceinline__ void tmem_st16u(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,"
+      "%15,%16};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
       : "memory");
 }
 
@@ -314,6 +343,12 @@ __device__ __forceinline__ bool named_bar_and(int id, int count, bool ok) {
 // Named barrier over `count` threads (a multiple of 32).
 __device__ __forceinline__ void named_bar(int id, int count) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
+// Arrive on a named barrier without waiting (the producer side of a producer/consumer pair whose
+// consumers use named_bar with the same id and count).
+__device__ __forceinline__ void named_bar_arrive(int id, int count) {
+  asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
 
 // Byte offset of element (row, col) of a [rows][64] 2-byte tile stored with the 128-byte swizzle

@@ -112,9 +112,13 @@ gdn_status gdn_causal_conv1d_silu(const void* x, gdn_dtype dtype, const float* w
  * final_state    : [N, Hv, dv, dk] fp32 or NULL (not written).  May not overlap initial_state.
  * cu_seqlens     : int32 [N+1] or NULL (then N == B).  Each sequence is chunked from its own
  *                  start; its last chunk may be partial.
- * workspace      : device scratch of at least gdn_chunk_fwd_workspace_size() bytes, 256-byte
- *                  aligned; holds the device status word (read it with gdn_workspace_status).
- *                  Contents on entry are ignored.  Concurrent calls need separate workspaces.
+ * workspace      : device scratch, 256-byte aligned, at least 256 bytes; its first word is the
+ *                  device status word (read it with gdn_workspace_status).  With at least
+ *                  gdn_chunk_fwd_workspace_size() bytes the bf16 d = 128 chunk-64 shape takes the
+ *                  fast two-kernel path, which keeps each chunk's state-independent operands
+ *                  there (about 16.5 KB per chunk and v-head); with less it takes a path that
+ *                  needs only the status word.  Contents on entry are ignored.  Concurrent calls
+ *                  need separate workspaces.
  * Supported: dk, dv in {16, 32, ..., 128} (multiples of 16), chunk in {16, 32, 64}.  The tensor-core
  * path (tcgen05 + TMA) serves dtype GDN_BF16, dk = dv = 128, chunk = 64; every other supported
  * shape runs on the CUDA-core path.  All pointers 16-byte aligned.
@@ -164,14 +168,16 @@ gdn_status gdn_chunk_fwd_strided(const void* q, int64_t q_tok_stride, const void
  * threads -- race on it: serialise them.  Device-detected faults land in that shared status word
  * and are not reported separately; use gdn_chunk_fwd with a workspace to read them.
  */
-#define GDN_NOALLOC_SCRATCH_BYTES (64 * 1024)
+#define GDN_NOALLOC_SCRATCH_BYTES (16 * 1024 * 1024)
 gdn_status gdn_chunk_fwd_noalloc(const void* q, const void* k, const void* v, const float* g,
                                  const float* beta, gdn_dtype dtype, float scale,
                                  const float* initial_state, const int32_t* cu_seqlens, int N,
                                  int B, int64_t T, int Hk, int Hv, int dk, int dv, int chunk,
                                  void* out, float* final_state, void* stream);
 
-/* Bytes of workspace gdn_chunk_fwd needs for these sizes (always > 0, a multiple of 256). */
+/* Bytes of workspace for gdn_chunk_fwd's fastest path at these sizes (always >= 256, a multiple of
+ * 256): ceil(B*T / 64) + N chunk slots x Hv x 16896 bytes + 1024 for the bf16 d = 128 chunk-64
+ * shape, 256 otherwise. */
 size_t gdn_chunk_fwd_workspace_size(int N, int B, int64_t T, int Hk, int Hv, int dk, int dv,
                                     int chunk);
 

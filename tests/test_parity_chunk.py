@@ -17,14 +17,20 @@ pytestmark = pytest.mark.gpu
 DEV = "cuda"
 
 
-def _gpu_chunk(x, g, beta, chunk, scale):
+def _gpu_chunk(x, g, beta, chunk, scale, workspace_bytes=None):
     cu = x["cu_seqlens"]
     S0 = x["initial_state"]
+    ws = None
+    if workspace_bytes is not None:
+        ws = torch.empty(workspace_bytes, dtype=torch.uint8, device=DEV)
     out, S = gdn.gdn_chunk_fwd(x["q"].to(DEV), x["k"].to(DEV), x["v"].to(DEV), g.to(DEV),
                                beta.to(DEV), scale=scale,
                                initial_state=None if S0 is None else S0.to(DEV),
-                               cu_seqlens=None if cu is None else cu.to(DEV), chunk=chunk)
+                               cu_seqlens=None if cu is None else cu.to(DEV), chunk=chunk,
+                               workspace=ws)
     torch.cuda.synchronize()
+    if ws is not None:
+        assert gdn.workspace_status(ws) == gdn.GDN_OK
     return out.cpu(), S.cpu()
 
 
@@ -79,6 +85,31 @@ def test_chunk_small_cases(case):
     out, S = _gpu_chunk(x, g, beta, chunk, dk ** -0.5)
     o_ref, S_ref = _full_oracle(x, g, beta, dk ** -0.5)
     _check(dtype, out, S, o_ref, S_ref, str(case))
+
+
+@pytest.mark.parametrize("case", [c for c in CASES if c[4] == c[5] == 128 and c[6] == 64
+                                  and c[7] == "bf16"])
+def test_chunk_small_workspace_path(case):
+    """The tensor-core shape with only the 256-byte status workspace: the path that keeps no
+    per-chunk operands in the workspace (one CTA pair per sequence and head)."""
+    B, T, Hk, Hv, dk, dv, chunk, dtype, seqlens, s0, a_mean = case
+    x = inputs.rule_inputs(B=B, T=T, Hk=Hk, Hv=Hv, dk=dk, dv=dv, dtype=dtype, seed=T + dk + 1,
+                           seqlens=seqlens, s0_std=s0, a_mean=a_mean)
+    g, beta = oracle_gates_f32(x)
+    out, S = _gpu_chunk(x, g, beta, chunk, dk ** -0.5, workspace_bytes=256)
+    o_ref, S_ref = _full_oracle(x, g, beta, dk ** -0.5)
+    _check(dtype, out, S, o_ref, S_ref, "small workspace " + str(case))
+
+
+def test_prefill_varlen_32k_small_workspace_path():
+    """The 32K varlen workload on the path without per-chunk workspace, every element."""
+    w = inputs.WORKLOADS["prefill_varlen_32k"]
+    x = inputs.rule_inputs(**w, seed=1000 + w["index"])
+    g, beta = oracle_gates_f32(x)
+    out, S = _gpu_chunk(x, g, beta, 64, 128 ** -0.5, workspace_bytes=256)
+    o_ref, S_ref = _full_oracle(x, g, beta, 128 ** -0.5)
+    assert_bf16_close(out, o_ref, "32k small-workspace path out")
+    assert_bf16_close(S, S_ref, "32k small-workspace path final states")
 
 
 def test_chunk_zero_decay():

@@ -33,9 +33,6 @@ def _noalloc(q, k, v, g, beta, S0, cu, chunk, out, S_T):
     assert st == gdn.GDN_OK, gdn.status_string(st)
 
 
-NOALLOC_SCRATCH_BYTES = 64 * 1024  # GDN_NOALLOC_SCRATCH_BYTES in include/gdn.h
-
-
 @pytest.mark.parametrize("chunk", [64, 32])
 def test_noalloc_matches_workspace_call_twice(chunk):
     x = inputs.rule_inputs(B=1, T=333, Hk=2, Hv=4, dk=128, dv=128, seed=77,
@@ -44,9 +41,10 @@ def test_noalloc_matches_workspace_call_twice(chunk):
     q, k, v = x["q"].to(DEV), x["k"].to(DEV), x["v"].to(DEV)
     g, beta = g.to(DEV), beta.to(DEV)
     S0, cu = x["initial_state"].to(DEV), x["cu_seqlens"].to(DEV)
-    # the reference call gets a caller workspace of the same size as the library's array, so both
-    # calls take the same kernel path and must agree bit for bit
-    ws = torch.empty(NOALLOC_SCRATCH_BYTES, dtype=torch.uint8, device=DEV)
+    # the reference call gets a caller workspace of gdn_chunk_fwd_workspace_size() bytes: both calls
+    # then take the same kernel path and must agree bit for bit
+    ws = torch.empty(gdn.workspace_size(4, 1, 333, 2, 4, 128, 128, chunk), dtype=torch.uint8,
+                     device=DEV)
     ref_out, ref_S = gdn.gdn_chunk_fwd(q, k, v, g, beta, initial_state=S0, cu_seqlens=cu,
                                        chunk=chunk, workspace=ws)
     assert gdn.workspace_status(ws) == gdn.GDN_OK
