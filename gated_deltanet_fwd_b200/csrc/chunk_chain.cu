@@ -91,6 +91,11 @@ struct ChainParams {
   int64_t gd_off;
   float scale;
   int N, Hk, Hv;
+  // intra-sequence scan (chunk_tm.cuh): phase 0 = one chain per sequence, 1 / 3 = scan phases
+  int phase;
+  int64_t lseg;     // segment length in tokens (0: no scan)
+  int64_t max_segs;
+  float* st;        // state arrays SOUT, BSEG, MSEG, SIN (scan phases only)
   int debug_skip_chunk;  // failure-test builds only: the producer withholds this chunk's tiles
   unsigned long long* trace;  // phase timing (trace builds only), else unused
 };
@@ -128,20 +133,46 @@ __global__ void __launch_bounds__(CH_THREADS, 1) chunk_chain_kernel(
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + SM_BAR + B_N * 8 + 4);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int n = blockIdx.x / P.Hv, h = blockIdx.x % P.Hv;
+  const int h = blockIdx.x % P.Hv;
   const int hk = h / (P.Hv / P.Hk);
-  const size_t sidx = ((size_t)n * P.Hv + h) * tm::D * tm::D;
 
-  int64_t s_beg, s_end, slot0;
-  if (!tm::seq_chunks(P.cu, P.T, n, s_beg, s_end, slot0)) {
-    if (tid == 0) report(P.status, GDN_ERR_DEVICE_ARG);
-    return;  // uniform across the CTA; nothing allocated yet
+  // ---- the unit this CTA runs: a whole sequence, or one segment of it (uniform across the CTA)
+  tm::Unit U;
+  {
+    bool bad = false;
+    if (!tm::find_unit(P.cu, P.T, P.N, P.lseg, P.phase, blockIdx.x / P.Hv, U, &bad)) {
+      if (bad && tid == 0) report(P.status, GDN_ERR_DEVICE_ARG);
+      return;  // nothing allocated yet
+    }
   }
+  const int n = U.n;
+  const int64_t s_beg = U.t_beg, s_end = U.t_end, slot0 = U.slot0;
+  const size_t hs = tm::STATE_FLOATS;
+  const size_t sidx = ((size_t)n * P.Hv + h) * hs;  // this sequence's state in S0 / S_T / SOUT
+  const size_t gidx = ((size_t)U.seg * P.Hv + h) * hs;  // this segment's state in BSEG/MSEG/SIN
+  float* const st_out = P.st;
+  float* const st_b = P.st + (size_t)P.N * P.Hv * hs;
+  float* const st_m = st_b + (size_t)P.max_segs * P.Hv * hs;
+  float* const st_in = st_m + (size_t)P.max_segs * P.Hv * hs;
+  // entry state (null: zero; the identity for a segment's transition) and where the leaving state
+  // goes (null: nowhere)
+  const bool ident = U.kind == tm::U_MSEG;
+  const float* src_state = U.kind == tm::U_MAIN0   ? (P.S0 ? P.S0 + sidx : nullptr)
+                           : U.kind == tm::U_MAINK ? st_in + gidx
+                                                   : nullptr;
+  float* dst_state = U.kind == tm::U_MAIN0   ? (U.nseg <= 1 ? (P.S_T ? P.S_T + sidx : nullptr)
+                                                            : st_out + sidx)
+                     : U.kind == tm::U_BSEG  ? st_b + gidx
+                     : U.kind == tm::U_MSEG  ? st_m + gidx
+                     : (U.k == U.nseg - 1 ? (P.S_T ? P.S_T + sidx : nullptr) : nullptr);
+  const bool has_out = U.kind == tm::U_MAIN0 || U.kind == tm::U_MAINK;
+  const bool zero_v = U.kind == tm::U_MSEG;  // the transition: the chain of v = 0 from the identity
+
   const int nchunks = (int)((s_end - s_beg + tm::C - 1) / tm::C);
   if (nchunks == 0) {  // empty sequence: the state passes through
-    if (P.S_T)
+    if (dst_state)
       for (int e = tid; e < tm::D * tm::D; e += CH_THREADS)
-        P.S_T[sidx + e] = P.S0 ? P.S0[sidx + e] : 0.0f;
+        dst_state[e] = src_state ? src_state[e] : 0.0f;
     return;
   }
 
@@ -195,7 +226,7 @@ __global__ void __launch_bounds__(CH_THREADS, 1) chunk_chain_kernel(
         const int32_t t0 = (int32_t)chunk_t0(c);
         unsigned char* sp = smem + st * STAGE;
         uint64_t* fb = &bars[B_FULL0 + st];
-        mbar_arrive_expect_tx(fb, STAGE_TX);
+        mbar_arrive_expect_tx(fb, zero_v ? STAGE_TX - 16384 : STAGE_TX);
 #ifdef GDN_FAULT_INJECTION
         if (c == P.debug_skip_chunk) continue;  // nothing lands: the waits on this stage run out
 #endif
@@ -203,8 +234,10 @@ __global__ void __launch_bounds__(CH_THREADS, 1) chunk_chain_kernel(
         tma_load_3d(sp + ST_KQ + 8192, &map_q, fb, 0, hk, t0);
         tma_load_3d(sp + ST_KQ + 16384, &map_k, fb, 64, hk, t0);
         tma_load_3d(sp + ST_KQ + 24576, &map_q, fb, 64, hk, t0);
-        tma_load_3d(sp + ST_V, &map_v, fb, 0, h, t0);
-        tma_load_3d(sp + ST_V + 8192, &map_v, fb, 64, h, t0);
+        if (!zero_v) {
+          tma_load_3d(sp + ST_V, &map_v, fb, 0, h, t0);
+          tma_load_3d(sp + ST_V + 8192, &map_v, fb, 64, h, t0);
+        }
         const int64_t slot = slot0 + c;
         tma_load_2d(sp + ST_TP, &map_tp, fb, 0, (int32_t)((slot * P.Hv + h) * 128));
         bulk_load(sp + ST_GD, P.ws + P.gd_off + ((size_t)slot * P.Hv + h) * tm::GD_BYTES,
@@ -246,9 +279,11 @@ __global__ void __launch_bounds__(CH_THREADS, 1) chunk_chain_kernel(
           mma_bf16_ts(tmem + TM_K, tmem + TM_SB + 8 * ks,
                       dadd(dKQ, (ks >> 2) * 16384 + (ks & 3) * 32), id_kq, ks > 0);
         mma_commit(&bars[B_K]);
+        if (!zero_v) {
 #pragma unroll
-        for (int ks = 0; ks < 4; ++ks)
-          mma_bf16_ss(tmem + TM_U, dadd(dVt, ks * 2048), dadd(dTp, ks * 32), id_v, ks > 0);
+          for (int ks = 0; ks < 4; ++ks)
+            mma_bf16_ss(tmem + TM_U, dadd(dVt, ks * 2048), dadd(dTp, ks * 32), id_v, ks > 0);
+        }
       }
       if (lane == 0) CH_TS(c, 2);
       __syncwarp();
@@ -258,7 +293,8 @@ __global__ void __launch_bounds__(CH_THREADS, 1) chunk_chain_kernel(
         tc_fence_after();
 #pragma unroll
         for (int ks = 0; ks < 4; ++ks)
-          mma_bf16_ts(tmem + TM_U, tmem + TM_X + 8 * ks, dadd(dTp, ks * 32), id_n64, 1);
+          mma_bf16_ts(tmem + TM_U, tmem + TM_X + 8 * ks, dadd(dTp, ks * 32), id_n64,
+                      !zero_v || ks > 0);
         mma_commit(&bars[B_U]);
       }
       __syncwarp();
@@ -270,10 +306,12 @@ __global__ void __launch_bounds__(CH_THREADS, 1) chunk_chain_kernel(
         for (int ks = 0; ks < 4; ++ks)
           mma_bf16_ts(tmem + TM_S, tmem + TM_UD + 8 * ks, dadd(dKn, ks * 2048), id_s, 1);
         mma_commit(&bars[B_S]);
+        if (has_out) {
 #pragma unroll
-        for (int ks = 0; ks < 4; ++ks)
-          mma_bf16_ts(tmem + TM_K, tmem + TM_UT + 8 * ks, dadd(dP, ks * 32), id_n64, ks > 0);
-        mma_commit(&bars[B_O]);
+          for (int ks = 0; ks < 4; ++ks)
+            mma_bf16_ts(tmem + TM_K, tmem + TM_UT + 8 * ks, dadd(dP, ks * 32), id_n64, ks > 0);
+          mma_commit(&bars[B_O]);
+        }
         mma_commit(&bars[B_EMPTY0 + st]);
       }
       __syncwarp();
@@ -289,7 +327,7 @@ __global__ void __launch_bounds__(CH_THREADS, 1) chunk_chain_kernel(
     const uint32_t lo = (uint32_t)(32 * warp) << 16;
     // initial state: fp32 master and bf16 operand copy
     {
-      const float* src = P.S0 ? P.S0 + sidx + (size_t)j * tm::D : nullptr;
+      const float* src = src_state ? src_state + (size_t)j * tm::D : nullptr;
 #pragma unroll
       for (int blk = 0; blk < 4; ++blk) {  // 32 columns at a time
         float v[32];
@@ -301,6 +339,10 @@ __global__ void __launch_bounds__(CH_THREADS, 1) chunk_chain_kernel(
           v[4 * q4 + 1] = f.y;
           v[4 * q4 + 2] = f.z;
           v[4 * q4 + 3] = f.w;
+        }
+        if (ident) {
+#pragma unroll
+          for (int q = 0; q < 32; ++q) v[q] = (32 * blk + q == j) ? 1.0f : 0.0f;
         }
         tmem_st16(tmem + lo + TM_S + 32 * blk, *reinterpret_cast<float(*)[16]>(v));
         tmem_st16(tmem + lo + TM_S + 32 * blk + 16, *reinterpret_cast<float(*)[16]>(v + 16));
@@ -435,7 +477,7 @@ __global__ void __launch_bounds__(CH_THREADS, 1) chunk_chain_kernel(
       // ---- outputs of chunk c: O^T = diag(Gamma) (S Q^T) + U^T P^T, held as scaled bf16 pairs
       // (rows 2q, 2q + 1) of value column j
       uint32_t ob[32];
-      const bool o_ok = wait(B_O, c & 1);
+      const bool o_ok = has_out && wait(B_O, c & 1);
       if (t4 == 0) CH_TS(c, 12);
       if (o_ok) {
         tc_fence_after();
@@ -492,10 +534,10 @@ __global__ void __launch_bounds__(CH_THREADS, 1) chunk_chain_kernel(
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp < 4 && P.S_T && !*abort_flag) {
+  if (warp < 4 && dst_state && !*abort_flag) {
     const int j = 32 * warp + lane;
     const uint32_t lo = (uint32_t)(32 * warp) << 16;
-    float* dst = P.S_T + sidx + (size_t)j * tm::D;
+    float* dst = dst_state + (size_t)j * tm::D;
 #pragma unroll
     for (int hh = 0; hh < 2; ++hh) {
       float v[64];
@@ -523,9 +565,12 @@ unsigned long long* g_chain_trace = nullptr;  // trace builds: device buffer of 
 cudaError_t launch_chunk_chain(const void* q, const void* k, const void* v, TokStrides ts,
                                float scale, const float* S0, const int32_t* cu, int N, int B,
                                int64_t T, int Hk, int Hv, void* out, float* S_T, void* ws,
-                               int* status, cudaStream_t s) {
+                               int phase, int64_t lseg, int* status, cudaStream_t s) {
   const int64_t n_tok = (int64_t)B * T;
-  const int64_t units = (int64_t)N * Hv;
+  const int64_t msegs = tm::max_segs(N, n_tok, lseg);
+  // units per v-head: phase 0 one per sequence; phase 1 at most one per sequence and two per
+  // segment; phase 3 at most one per segment
+  const int64_t units = (phase == 0 ? (int64_t)N : phase == 1 ? N + 2 * msegs : msegs) * Hv;
   if (units == 0) return cudaSuccess;
   if (units > 0x7fffffff) return cudaErrorInvalidConfiguration;
   const int64_t slots = tm::max_slots(N, n_tok);
@@ -549,6 +594,11 @@ cudaError_t launch_chunk_chain(const void* q, const void* k, const void* v, TokS
   p.N = N;
   p.Hk = Hk;
   p.Hv = Hv;
+  p.phase = phase;
+  p.lseg = phase == 0 ? 0 : lseg;
+  p.max_segs = msegs;
+  p.st = phase == 0 ? nullptr
+                    : reinterpret_cast<float*>(wsb + tm::states_offset(N, n_tok, Hv));
   p.debug_skip_chunk = g_debug_skip_chunk;
   p.trace = g_chain_trace;
   static bool attr_set = false;  // idempotent attribute; a benign race between host threads

@@ -23,6 +23,15 @@ inline bool ptr_ok(const void* p) { return p != nullptr && aligned16(p); }
 
 constexpr size_t kStatusBytes = 256;  // status word + padding to keep the workspace aligned
 
+// SM count of the current device (148 if it cannot be read): sets the scan's segment length
+int sm_count() {
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return 148;
+  return sms;
+}
+
 }  // namespace
 
 extern "C" {
@@ -100,8 +109,12 @@ gdn_status gdn_causal_conv1d_silu(const void* x, gdn_dtype dtype, const float* w
 size_t gdn_chunk_fwd_workspace_size(int N, int B, int64_t T, int Hk, int Hv, int dk, int dv,
                                     int chunk) {
   (void)Hk;
-  if (dk == gdn::tm::D && dv == gdn::tm::D && chunk == gdn::tm::C && N >= 0 && B >= 0 && T >= 0 && Hv >= 1)
-    return (gdn::tm::workspace_bytes(N, (int64_t)B * T, Hv) + 255) & ~size_t(255);
+  if (dk == gdn::tm::D && dv == gdn::tm::D && chunk == gdn::tm::C && N >= 0 && B >= 0 && T >= 0 &&
+      Hv >= 1) {
+    const int64_t n_tok = (int64_t)B * T;
+    const int64_t lseg = gdn::tm::scan_segment_tokens(n_tok, Hv, sm_count());
+    return (gdn::tm::workspace_bytes_scan(N, n_tok, Hv, lseg) + 255) & ~size_t(255);
+  }
   return kStatusBytes;
 }
 
@@ -157,12 +170,26 @@ gdn_status gdn_chunk_fwd_strided(const void* q, int64_t q_tok_stride, const void
   const TokStrides ts{q_tok_stride, k_tok_stride, v_tok_stride};
   cudaError_t e;
   if (dtype == GDN_BF16 && dk == gdn::tm::D && dv == gdn::tm::D && chunk == gdn::tm::C) {
-    if (workspace_bytes >= gdn::tm::workspace_bytes(N, (int64_t)B * T, Hv)) {
-      // prep kernel over all (chunk, k-head), then the chain over (sequence, v-head)
+    const int64_t n_tok = (int64_t)B * T;
+    const int64_t lseg = gdn::tm::scan_segment_tokens(n_tok, Hv, sm_count());
+    if (lseg > 0 && workspace_bytes >= gdn::tm::workspace_bytes_scan(N, n_tok, Hv, lseg)) {
+      // prep over all (chunk, k-head); chains of segment 0 and the middle segments' maps; the
+      // prefix over segments; chains of the later segments from their entry states
       e = launch_chunk_prep(q, k, ts, g, beta, cu_seqlens, N, B, T, Hk, Hv, workspace, status, s);
       if (e == cudaSuccess)
         e = launch_chunk_chain(q, k, v, ts, scale, initial_state, cu_seqlens, N, B, T, Hk, Hv,
-                               out, final_state, workspace, status, s);
+                               out, final_state, workspace, 1, lseg, status, s);
+      if (e == cudaSuccess)
+        e = launch_scan_prefix(cu_seqlens, N, B, T, Hv, lseg, workspace, status, s);
+      if (e == cudaSuccess)
+        e = launch_chunk_chain(q, k, v, ts, scale, initial_state, cu_seqlens, N, B, T, Hk, Hv,
+                               out, final_state, workspace, 3, lseg, status, s);
+    } else if (workspace_bytes >= gdn::tm::workspace_bytes(N, n_tok, Hv)) {
+      // prep over all (chunk, k-head), then one chain per (sequence, v-head)
+      e = launch_chunk_prep(q, k, ts, g, beta, cu_seqlens, N, B, T, Hk, Hv, workspace, status, s);
+      if (e == cudaSuccess)
+        e = launch_chunk_chain(q, k, v, ts, scale, initial_state, cu_seqlens, N, B, T, Hk, Hv,
+                               out, final_state, workspace, 0, 0, status, s);
     } else {
       e = launch_chunk_tc(q, k, v, ts, g, beta, scale, initial_state, cu_seqlens, N, B, T, Hk,
                           Hv, out, final_state, status, s);

@@ -174,10 +174,15 @@ bool make_rows64_map(CUtensorMap* m, const void* base, int64_t rows, uint32_t bo
 cudaError_t launch_chunk_prep(const void* q, const void* k, TokStrides ts, const float* g,
                               const float* beta, const int32_t* cu, int N, int B, int64_t T,
                               int Hk, int Hv, void* ws, int* status, cudaStream_t s);
+// phase 0: one chain per (sequence, v-head); phases 1 and 3 (with launch_scan_prefix between
+// them): the intra-sequence scan with segments of lseg tokens (chunk_tm.cuh), for which `ws` holds
+// at least tm::workspace_bytes_scan(N, B*T, Hv, lseg) bytes.
 cudaError_t launch_chunk_chain(const void* q, const void* k, const void* v, TokStrides ts,
                                float scale, const float* S0, const int32_t* cu, int N, int B,
                                int64_t T, int Hk, int Hv, void* out, float* S_T, void* ws,
-                               int* status, cudaStream_t s);
+                               int phase, int64_t lseg, int* status, cudaStream_t s);
+cudaError_t launch_scan_prefix(const int32_t* cu, int N, int B, int64_t T, int Hv, int64_t lseg,
+                               void* ws, int* status, cudaStream_t s);
 
 // Tensor-core chunk path without scratch (one CTA pair per sequence and head): bf16,
 // dk = dv = 128, chunk = 64.

@@ -112,6 +112,42 @@ def test_prefill_varlen_32k_small_workspace_path():
     assert_bf16_close(S, S_ref, "32k small-workspace path final states")
 
 
+def _no_scan_workspace_bytes(N, n_tok, Hv):
+    """Workspace with room for the per-chunk operands but not for the scan's state arrays: the
+    tensor-core path then runs one chain per (sequence, v-head).  Layout as in the library:
+    1024 header bytes + (ceil(n_tok / 64) + N) chunk slots x Hv x (16384 + 512) bytes."""
+    return 1024 + (-(-n_tok // 64) + N) * Hv * (16384 + 512)
+
+
+SCAN_CASES = [
+    # T, seqlens, Hk, Hv, s0, a_mean, zero_g
+    (3000, None, 1, 2, 0.02, -6.0, False),          # one sequence, six segments
+    (3000, None, 1, 2, 0.02, 0.0, True),            # g = 0: the state carries through every segment
+    (4300, [1500, 100, 0, 2600, 100], 2, 4, 0.05, -3.0, False),  # varlen: split and unsplit
+    (2049, None, 1, 1, None, -6.0, False),          # Hk = Hv, zero initial state, ragged tail
+]
+
+
+@pytest.mark.parametrize("case", SCAN_CASES)
+def test_chunk_intra_sequence_scan(case):
+    """Sequences longer than two segments run as the intra-sequence scan (segment 0 and the middle
+    segments' affine maps in parallel, a prefix over the maps, then the later segments from their
+    entry states); against the oracle, and against the same call without the scan."""
+    T, seqlens, Hk, Hv, s0, a_mean, zero_g = case
+    x = inputs.rule_inputs(B=1, T=T, Hk=Hk, Hv=Hv, dk=128, dv=128, dtype="bf16", seed=T + Hv,
+                           seqlens=seqlens, s0_std=s0, a_mean=a_mean)
+    g, beta = oracle_gates_f32(x)
+    if zero_g:
+        g = torch.zeros_like(g)
+    N = x["N"]
+    out, S = _gpu_chunk(x, g, beta, 64, 128 ** -0.5)
+    o_ref, S_ref = _full_oracle(x, g, beta, 128 ** -0.5)
+    _check("bf16", out, S, o_ref, S_ref, "scan " + str(case))
+    out1, S1 = _gpu_chunk(x, g, beta, 64, 128 ** -0.5,
+                          workspace_bytes=_no_scan_workspace_bytes(N, T, Hv))
+    _check("bf16", out1, S1, o_ref, S_ref, "one chain " + str(case))
+
+
 def test_chunk_zero_decay():
     """g = 0 (no forgetting): nothing damps an error carried between chunks."""
     x = inputs.rule_inputs(B=1, T=256, Hk=1, Hv=2, dk=128, dv=128, seed=4, s0_std=0.02)
