@@ -357,6 +357,51 @@ def bench_decode(dist, gdn, K, W, peaks):
                 gpu_launches=2 * steps * K)
 
 
+def bench_decode_layer(dist, gdn, K, W, peaks):
+    """The decode workload's shapes with one token of the whole layer core per launch
+    (gdn_decode_layer_step: conv with the cached history, gates, recurrent step, gated RMSNorm);
+    one step = 64 consecutive tokens."""
+    w = inputs.WORKLOADS["decode_layer_256"]
+    steps = w["steps"]
+    x = inputs.decode_layer_inputs(**w, seed=1000 + w["index"])
+    dev = torch.device("cuda", torch.cuda.current_device())
+    N, Hk, Hv, dk, dv, Kc = w["N"], w["Hk"], w["Hv"], w["dk"], w["dv"], w["K"]
+    C = x["C"]
+    state = x["state"].to(dev)
+    cs = [x["conv_state"].to(dev), torch.empty_like(x["conv_state"]).to(dev)]
+    conv_w, A_log, dt_bias = x["conv_w"].to(dev), x["A_log"].to(dev), x["dt_bias"].to(dev)
+    norm_w = x["norm_w"].to(dev)
+    mix = [t.to(dev) for t in x["mix"]]
+    a = [t.to(dev) for t in x["a"]]
+    b = [t.to(dev) for t in x["b"]]
+    z = [t.to(dev) for t in x["z"]]
+    y = torch.empty(N, Hv, dv, dtype=torch.bfloat16, device=dev)
+    kt = KernelTimer()
+
+    def step(timed):
+        for s_ in range(steps):
+            call = lambda: gdn.gdn_decode_layer_step(mix[s_], a[s_], b[s_], z[s_], conv_w,
+                                                     cs[s_ & 1], cs[(s_ + 1) & 1], A_log,
+                                                     dt_bias, norm_w, state, Hk, y=y)
+            kt(call) if timed else call()
+
+    ms = timed_region(dist, step, K, W)
+    k_ms = kt.mean_ms()
+    state_bytes = N * Hv * dv * dk * 4
+    hist_bytes = N * C * (Kc - 1) * 4
+    io_bytes = (N * C + 2 * N * Hv + 2 * N * Hv * dv) * 2  # mix, a, b, z in; y out (bf16)
+    bytes_per_launch = 2 * state_bytes + 2 * hist_bytes + io_bytes
+    achieved = bytes_per_launch / (k_ms * 1e-3) / 1e9
+    return dict(value=N * steps * K * dist.world / (ms * 1e-3), unit="seqs/s",
+                ms_per_step=ms / K, token_us=k_ms * 1e3,
+                roofline=dict(bound="hbm", kernel="gdn_decode_layer_step", achieved=achieved,
+                              peak=peaks["hbm"], unit="GB/s", frac=achieved / peaks["hbm"],
+                              frac_of_nominal_8tbs=achieved / 8000.0,
+                              bytes_per_launch=bytes_per_launch,
+                              peak_source=peaks["source"] + " HBM copy"),
+                gpu_launches=steps * K)
+
+
 def bench_layer_core(dist, gdn, K, W, peaks):
     w = inputs.WORKLOADS["layer_core_2x16k"]
     x = inputs.layer_core_inputs(**w, seed=1000 + w["index"])
@@ -537,6 +582,9 @@ def main():
     dec = bench_decode(dist, gdn, max(2, args.steps // 4), args.warmup, peaks)
     dec["clocks"] = clocks.stop()
     clocks.start()
+    dec_layer = bench_decode_layer(dist, gdn, max(2, args.steps // 4), args.warmup, peaks)
+    dec_layer["clocks"] = clocks.stop()
+    clocks.start()
     core = bench_layer_core(dist, gdn, max(2, args.steps // 4), args.warmup, peaks)
     core["clocks"] = clocks.stop()
     cpu = None
@@ -554,7 +602,8 @@ def main():
                                 l2="inputs larger than L2 (no flush)",
                                 parallelism=f"replica x{dist.world}"),
                     roofline=pre["roofline"], e2e=pre["e2e"], gpu_launches=pre["gpu_launches"],
-                    clocks=clk, cpu_baseline=cpu, decode=dec, layer_core=core)
+                    clocks=clk, cpu_baseline=cpu, decode=dec, decode_layer=dec_layer,
+                    layer_core=core)
         print(json.dumps(line), flush=True)
     dist.close()
     return 0

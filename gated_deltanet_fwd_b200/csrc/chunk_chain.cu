@@ -93,7 +93,7 @@ struct ChainParams {
   int N, Hk, Hv;
   // intra-sequence scan (chunk_tm.cuh): phase 0 = one chain per sequence, 1 / 3 = scan phases
   int phase;
-  int64_t lseg;     // segment length in tokens (0: no scan)
+  const int64_t* plan;  // segment length in tokens chosen on the device (0: no scan); scan only
   int64_t max_segs;
   float* st;        // state arrays SOUT, BSEG, MSEG, SIN (scan phases only)
   int debug_skip_chunk;  // failure-test builds only: the producer withholds this chunk's tiles
@@ -140,7 +140,8 @@ __global__ void __launch_bounds__(CH_THREADS, 1) chunk_chain_kernel(
   tm::Unit U;
   {
     bool bad = false;
-    if (!tm::find_unit(P.cu, P.T, P.N, P.lseg, P.phase, blockIdx.x / P.Hv, U, &bad)) {
+    const int64_t lseg = P.phase == 0 ? 0 : *P.plan;
+    if (!tm::find_unit(P.cu, P.T, P.N, lseg, P.phase, blockIdx.x / P.Hv, U, &bad)) {
       if (bad && tid == 0) report(P.status, GDN_ERR_DEVICE_ARG);
       return;  // nothing allocated yet
     }
@@ -244,12 +245,11 @@ __global__ void __launch_bounds__(CH_THREADS, 1) chunk_chain_kernel(
                   tm::GD_BYTES, fb);
         issued = c + 1;
       }
-      // never leave the CTA with copies still landing in shared memory
+      // never leave the CTA with copies still landing in shared memory (each wait bounded; a
+      // stage whose copies were never issued simply runs out)
       for (int c = issued - 2 < 0 ? 0 : issued - 2; c < issued; ++c)
-        if (!mbar_wait(&bars[B_FULL0 + (c & 1)], (uint32_t)(c >> 1) & 1)) {
+        if (!mbar_wait(&bars[B_FULL0 + (c & 1)], (uint32_t)(c >> 1) & 1))
           report(P.status, GDN_ERR_TIMEOUT);
-          break;
-        }
     }
   } else if (warp == W_MMA) {
     // ------------------------------------------------------------ MMA issuer ---------------
@@ -567,7 +567,7 @@ cudaError_t launch_chunk_chain(const void* q, const void* k, const void* v, TokS
                                int64_t T, int Hk, int Hv, void* out, float* S_T, void* ws,
                                int phase, int64_t lseg, int* status, cudaStream_t s) {
   const int64_t n_tok = (int64_t)B * T;
-  const int64_t msegs = tm::max_segs(N, n_tok, lseg);
+  const int64_t msegs = tm::max_segs(N, n_tok, lseg);  // lseg: the smallest the planner may pick
   // units per v-head: phase 0 one per sequence; phase 1 at most one per sequence and two per
   // segment; phase 3 at most one per segment
   const int64_t units = (phase == 0 ? (int64_t)N : phase == 1 ? N + 2 * msegs : msegs) * Hv;
@@ -595,7 +595,7 @@ cudaError_t launch_chunk_chain(const void* q, const void* k, const void* v, TokS
   p.Hk = Hk;
   p.Hv = Hv;
   p.phase = phase;
-  p.lseg = phase == 0 ? 0 : lseg;
+  p.plan = reinterpret_cast<const int64_t*>(wsb + tm::PLAN_OFF);
   p.max_segs = msegs;
   p.st = phase == 0 ? nullptr
                     : reinterpret_cast<float*>(wsb + tm::states_offset(N, n_tok, Hv));

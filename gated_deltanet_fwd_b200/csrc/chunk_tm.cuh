@@ -4,7 +4,8 @@
 // (chunk_chain.cu) streams them in with TMA while it carries the state from chunk to chunk.
 //
 // Workspace (from its 256-byte-aligned base):
-//   [0, 1024)                 status word (first int) and padding
+//   [0, 1024)                 status word (first int), the scan's segment length (int64 at byte
+//                             8, written on the device by the planner), padding
 //   TP  [slots][Hv][128][64]  bf16: rows 0..63 T' = (I + A)^{-1} diag(beta), rows 64..127 the
 //                             decay-masked P = e^{gamma_r - gamma_s} q_r.k_s (s <= r); rows are
 //                             128 bytes, loaded by the chain as one 128-byte-swizzled tile
@@ -43,6 +44,7 @@ constexpr int D = 128;                 // dk = dv
 constexpr uint32_t TP_BYTES = 16384;   // [T'; P] per (slot, v-head)
 constexpr uint32_t GD_BYTES = 512;     // Gamma, d per (slot, v-head)
 constexpr size_t HEADER_BYTES = 1024;  // status word + padding
+constexpr size_t PLAN_OFF = 8;         // int64 segment length chosen for the call (0: no scan)
 
 __host__ __device__ inline int64_t max_slots(int N, int64_t n_tok) {
   return (n_tok + C - 1) / C + N;
@@ -109,56 +111,71 @@ struct Unit {
   int64_t seg;           // global segment index (n, k)
 };
 
-// Unit `u` (index among the units of `phase`, per v-head).  Returns false past the last unit, or
-// with *bad set for a malformed cu_seqlens met on the way (nothing may be read through it then).
-// O(N) reads of cu_seqlens.
+// Longest-first order of a phase's units, so that the hardware's in-order block dispatch packs
+// them well: rank 0 = whole sequences longer than one segment, 1 = full-length segments and the
+// middle segments' maps, 2 = the rest.  Phase 0 (no scan) keeps sequence order.
+__host__ __device__ inline int unit_rank(int phase, int kind, int64_t k, int64_t nseg, int64_t len,
+                                         int64_t lseg) {
+  if (phase == 0) return 0;
+  if (kind == U_MAIN0 && nseg <= 1) return len > lseg ? 0 : 2;
+  if (kind == U_MAINK && k == nseg - 1) return len - k * lseg == lseg ? 1 : 2;
+  return 1;
+}
+
+// Unit `u` (index among the units of `phase`, per v-head, in longest-first order).  Returns false
+// past the last unit, or with *bad set for a malformed cu_seqlens met on the way (nothing may be
+// read through it then).  O(N) reads of cu_seqlens per rank.
 __device__ inline bool find_unit(const int32_t* cu, int64_t T, int N, int64_t lseg, int phase,
                                  int64_t u, Unit& out, bool* bad) {
   *bad = false;
-  int64_t slot_base = 0, seg_base = 0;
-  for (int m = 0; m < N; ++m) {
-    int64_t a, b;
-    if (cu) {
-      a = cu[m];
-      b = cu[m + 1];
-      if (a < 0 || b < a || b > T) {
-        *bad = true;
-        return false;
-      }
-    } else {
-      a = (int64_t)m * T;
-      b = a + T;
-    }
-    const int64_t len = b - a;
-    const int64_t nseg = seg_count(len, lseg);
-    const int64_t nu = units_of(phase, nseg);
-    if (u < nu) {
-      int64_t k;
-      int kind;
-      if (phase == 3) {
-        k = u + 1;
-        kind = U_MAINK;
-      } else if (u == 0) {
-        k = 0;
-        kind = U_MAIN0;
+  for (int rank = 0; rank < 3; ++rank) {
+    int64_t slot_base = 0, seg_base = 0;
+    for (int m = 0; m < N; ++m) {
+      int64_t a, b;
+      if (cu) {
+        a = cu[m];
+        b = cu[m + 1];
+        if (a < 0 || b < a || b > T) {
+          *bad = true;
+          return false;
+        }
       } else {
-        k = 1 + (u - 1) / 2;
-        kind = ((u - 1) & 1) ? U_MSEG : U_BSEG;
+        a = (int64_t)m * T;
+        b = a + T;
       }
-      const int64_t span = nseg <= 1 ? len : lseg;
-      out.n = m;
-      out.kind = kind;
-      out.k = k;
-      out.nseg = nseg;
-      out.t_beg = a + k * span;
-      out.t_end = out.t_beg + span < b ? out.t_beg + span : b;
-      out.slot0 = slot_base + k * (span / C);
-      out.seg = seg_base + k;
-      return true;
+      const int64_t len = b - a;
+      const int64_t nseg = seg_count(len, lseg);
+      const int64_t nu = units_of(phase, nseg);
+      for (int64_t i = 0; i < nu; ++i) {
+        int64_t k;
+        int kind;
+        if (phase == 3) {
+          k = i + 1;
+          kind = U_MAINK;
+        } else if (i == 0) {
+          k = 0;
+          kind = U_MAIN0;
+        } else {
+          k = 1 + (i - 1) / 2;
+          kind = ((i - 1) & 1) ? U_MSEG : U_BSEG;
+        }
+        if (unit_rank(phase, kind, k, nseg, len, lseg) != rank) continue;
+        if (u-- > 0) continue;
+        const int64_t span = nseg <= 1 ? len : lseg;
+        out.n = m;
+        out.kind = kind;
+        out.k = k;
+        out.nseg = nseg;
+        out.t_beg = a + k * span;
+        out.t_end = out.t_beg + span < b ? out.t_beg + span : b;
+        out.slot0 = slot_base + k * (span / C);
+        out.seg = seg_base + k;
+        return true;
+      }
+      slot_base += (len + C - 1) / C;
+      seg_base += nseg;
     }
-    u -= nu;
-    slot_base += (len + C - 1) / C;
-    seg_base += nseg;
+    if (phase == 0) break;
   }
   return false;
 }

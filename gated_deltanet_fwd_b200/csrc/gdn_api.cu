@@ -171,11 +171,16 @@ gdn_status gdn_chunk_fwd_strided(const void* q, int64_t q_tok_stride, const void
   cudaError_t e;
   if (dtype == GDN_BF16 && dk == gdn::tm::D && dv == gdn::tm::D && chunk == gdn::tm::C) {
     const int64_t n_tok = (int64_t)B * T;
-    const int64_t lseg = gdn::tm::scan_segment_tokens(n_tok, Hv, sm_count());
+    const int sms = sm_count();
+    const int64_t lseg = gdn::tm::scan_segment_tokens(n_tok, Hv, sms);
     if (lseg > 0 && workspace_bytes >= gdn::tm::workspace_bytes_scan(N, n_tok, Hv, lseg)) {
-      // prep over all (chunk, k-head); chains of segment 0 and the middle segments' maps; the
-      // prefix over segments; chains of the later segments from their entry states
-      e = launch_chunk_prep(q, k, ts, g, beta, cu_seqlens, N, B, T, Hk, Hv, workspace, status, s);
+      // the planner picks the segment length (or none); prep over all (chunk, k-head); chains of
+      // segment 0 and the middle segments' maps; the prefix over segments; chains of the later
+      // segments from their entry states
+      e = launch_scan_plan(cu_seqlens, N, B, T, Hv, sms, lseg, workspace, status, s);
+      if (e == cudaSuccess)
+        e = launch_chunk_prep(q, k, ts, g, beta, cu_seqlens, N, B, T, Hk, Hv, workspace, status,
+                              s);
       if (e == cudaSuccess)
         e = launch_chunk_chain(q, k, v, ts, scale, initial_state, cu_seqlens, N, B, T, Hk, Hv,
                                out, final_state, workspace, 1, lseg, status, s);
@@ -225,6 +230,34 @@ gdn_status gdn_recurrent_step(const void* q, const void* k, const void* v, const
     return GDN_ERR_INVALID_ARG;
   return from_cuda(launch_recurrent(q, k, v, g, beta, dtype, scale, state, N, Hk, Hv, dk, dv, out,
                                     as_stream(stream)));
+}
+
+gdn_status gdn_decode_layer_step(const void* mix, const void* a, const void* b, const void* z,
+                                 gdn_dtype dtype, const float* conv_w, const float* conv_bias,
+                                 int K, const float* conv_state_in, float* conv_state_out,
+                                 const float* A_log, const float* dt_bias, const float* norm_w,
+                                 float l2_eps, float norm_eps, float scale, float* state, int N,
+                                 int Hk, int Hv, int dk, int dv, void* y, void* stream) {
+  if (bad_dtype(dtype) || N < 0 || Hk < 1 || Hv < 1 || dk < 1 || dv < 1 || K < 1)
+    return GDN_ERR_INVALID_ARG;
+  if (Hv % Hk != 0) return GDN_ERR_INVALID_ARG;
+  if (!(scale == scale) || !(l2_eps >= 0.0f) || !(norm_eps >= 0.0f)) return GDN_ERR_INVALID_ARG;
+  if (dk != 128 || dv != 128 || K > 8) return GDN_ERR_UNSUPPORTED;
+  if (N == 0) return GDN_OK;
+  if (!ptr_ok(mix) || !a || !b || !ptr_ok(z) || !conv_w || !A_log || !dt_bias || !norm_w ||
+      !ptr_ok(state) || !ptr_ok(y))
+    return GDN_ERR_INVALID_ARG;
+  const size_t C = 2 * (size_t)Hk * dk + (size_t)Hv * dv;
+  if (K > 1) {
+    if (!conv_state_in || !conv_state_out) return GDN_ERR_INVALID_ARG;
+    const size_t bytes = (size_t)N * C * (K - 1) * sizeof(float);
+    const char* i0 = (const char*)conv_state_in;
+    const char* o0 = (const char*)conv_state_out;
+    if (i0 < o0 + bytes && o0 < i0 + bytes) return GDN_ERR_INVALID_ARG;
+  }
+  return from_cuda(launch_decode_fused(mix, a, b, z, dtype, conv_w, conv_bias, K, conv_state_in,
+                                       conv_state_out, A_log, dt_bias, norm_w, l2_eps, norm_eps,
+                                       scale, state, N, Hk, Hv, y, as_stream(stream)));
 }
 
 gdn_status gdn_gated_rmsnorm(const void* x, const void* z, gdn_dtype dtype, const float* w,

@@ -150,6 +150,13 @@ cudaError_t launch_recurrent(const void* q, const void* k, const void* v, const 
                              const float* beta, gdn_dtype dt, float scale, float* state, int N,
                              int Hk, int Hv, int dk, int dv, void* out, cudaStream_t s);
 
+cudaError_t launch_decode_fused(const void* mix, const void* a, const void* b, const void* z,
+                                gdn_dtype dt, const float* conv_w, const float* conv_bias, int K,
+                                const float* cs_in, float* cs_out, const float* A_log,
+                                const float* dt_bias, const float* norm_w, float l2_eps,
+                                float norm_eps, float scale, float* state, int N, int Hk, int Hv,
+                                void* y, cudaStream_t s);
+
 // Element distances between consecutive tokens of q, k and v (dense: Hk*dk, Hk*dk, Hv*dv).
 struct TokStrides {
   int64_t q, k, v;
@@ -181,6 +188,10 @@ cudaError_t launch_chunk_chain(const void* q, const void* k, const void* v, TokS
                                float scale, const float* S0, const int32_t* cu, int N, int B,
                                int64_t T, int Hk, int Hv, void* out, float* S_T, void* ws,
                                int phase, int64_t lseg, int* status, cudaStream_t s);
+// One-thread planner: writes the call's segment length (0, lseg, 2 lseg or 4 lseg) into the
+// workspace for the two chain phases and the prefix to read.
+cudaError_t launch_scan_plan(const int32_t* cu, int N, int B, int64_t T, int Hv, int sms,
+                             int64_t lseg, void* ws, int* status, cudaStream_t s);
 cudaError_t launch_scan_prefix(const int32_t* cu, int N, int B, int64_t T, int Hv, int64_t lseg,
                                void* ws, int* status, cudaStream_t s);
 

@@ -40,6 +40,8 @@ SIGNATURES = {
     "gdn_workspace_status": (_I, [_P, _P, ctypes.POINTER(_I)]),
     "gdn_recurrent_step": (_I, [_P, _P, _P, _P, _P, _I, _F, _P, _I, _I, _I, _I, _I, _P, _P]),
     "gdn_gated_rmsnorm": (_I, [_P, _P, _I, _P, _F, _I64, _I, _P, _P]),
+    "gdn_decode_layer_step": (_I, [_P, _P, _P, _P, _I, _P, _P, _I, _P, _P, _P, _P, _P, _F, _F, _F,
+                                   _P, _I, _I, _I, _I, _I, _P, _P]),
 }
 
 _lib = None
@@ -201,6 +203,27 @@ def gdn_recurrent_step(q, k, v, g, beta, state, scale=None, out=None):
         _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _dt(q), float(scale), _ptr(state), N, Hk,
         Hv, dk, dv, _ptr(out), _stream(q)))
     return out
+
+
+def gdn_decode_layer_step(mix, a, b, z, conv_w, conv_state_in, conv_state_out, A_log, dt_bias,
+                          norm_w, state, Hk, conv_bias=None, l2_eps=1e-6, norm_eps=1e-6,
+                          scale=None, y=None):
+    """One decode token of the layer core: conv (history in conv_state_in, advanced into
+    conv_state_out) + SiLU + q/k L2 norm, gates, recurrent step on `state` (in place), gated
+    RMSNorm with z.  mix: [N, C]; a, b: [N, Hv]; z: [N, Hv, dv]; returns y [N, Hv, dv]."""
+    _cuda(mix, a, b, z, conv_w, conv_bias, conv_state_in, conv_state_out, A_log, dt_bias, norm_w,
+          state, y)
+    N, Hv, dv = z.shape
+    dk = state.shape[3]
+    K = conv_w.shape[1]
+    scale = dk ** -0.5 if scale is None else scale
+    y = torch.empty_like(z) if y is None else y
+    _check("gdn_decode_layer_step", load().gdn_decode_layer_step(
+        _ptr(mix), _ptr(a), _ptr(b), _ptr(z), _dt(mix), _ptr(conv_w), _ptr(conv_bias), K,
+        _ptr(conv_state_in), _ptr(conv_state_out), _ptr(A_log), _ptr(dt_bias), _ptr(norm_w),
+        float(l2_eps), float(norm_eps), float(scale), _ptr(state), N, Hk, Hv, dk, dv, _ptr(y),
+        _stream(mix)))
+    return y
 
 
 def gdn_gated_rmsnorm(x, z, w, eps=1e-6, y=None):

@@ -32,6 +32,9 @@ WORKLOADS = {
                        s0_std=0.02),
     "layer_core_2x16k": dict(index=4, B=2, T=16384, Hk=16, Hv=32, dk=128, dv=128,
                              dtype="bf16", chunk=64, K=4, eps=1e-6),
+    # the decode workload's shapes, one token of the whole layer core per step
+    "decode_layer_256": dict(index=3, N=256, Hk=16, Hv=32, dk=128, dv=128, dtype="bf16",
+                             steps=64, K=4, s0_std=0.02, eps=1e-6),
 }
 
 
@@ -112,6 +115,35 @@ def decode_inputs(*, N, Hk, Hv, dk, dv, dtype="bf16", seed=0, steps=1, s0_std=0.
         as_.append(_randn(gen, (N, Hv)))
         bs.append(_randn(gen, (N, Hv)))
     return dict(state=state, q=qs, k=ks, v=vs, a=as_, b=bs, A_log=A_log, dt_bias=dt_bias)
+
+
+def decode_layer_inputs(*, N, Hk, Hv, dk, dv, K=4, dtype="bf16", seed=0, steps=1, s0_std=0.02,
+                        **_unused):
+    """Inputs of `steps` decode tokens of the whole layer core for N sequences.
+
+    Per step: mix [N, C] (the token's [q | k | v] projections before the conv), a, b [N, Hv] and
+    z [N, Hv, dv], all in ``dtype`` and ~ N(0, 1).  Once: conv_w [C, K] ~ U(+-1/sqrt(K)); the conv
+    history conv_state [N, C, K-1] (fp32 holding bf16-rounded N(0, 1) values, like past inputs);
+    A_log, dt_bias [Hv]; norm_w [dv] ~ N(0, 0.02); state [N, Hv, dv, dk] ~ N(0, s0_std).
+    """
+    gen = _gen(seed)
+    dt = torch_dtype(dtype)
+    C = 2 * Hk * dk + Hv * dv
+    bound = 1.0 / math.sqrt(K)
+    conv_w = (torch.rand(C, K, generator=gen, dtype=torch.float32) * 2.0 - 1.0) * bound
+    conv_state = _randn(gen, (N, C, K - 1)).to(dt).float()
+    A_log = torch.log(torch.rand(Hv, generator=gen, dtype=torch.float32) * 15.0 + 1.0)
+    dt_bias = _randn(gen, (Hv,), std=0.1)
+    norm_w = _randn(gen, (dv,), std=0.02)
+    state = _randn(gen, (N, Hv, dv, dk), std=s0_std)
+    mix, a, b, z = [], [], [], []
+    for _ in range(steps):
+        mix.append(_randn(gen, (N, C)).to(dt))
+        a.append(_randn(gen, (N, Hv)).to(dt))
+        b.append(_randn(gen, (N, Hv)).to(dt))
+        z.append(_randn(gen, (N, Hv, dv)).to(dt))
+    return dict(mix=mix, a=a, b=b, z=z, conv_w=conv_w, conv_state=conv_state, A_log=A_log,
+                dt_bias=dt_bias, norm_w=norm_w, state=state, C=C)
 
 
 def layer_core_inputs(*, B, T, Hk, Hv, dk, dv, K=4, dtype="bf16", seed=0, seqlens=None,

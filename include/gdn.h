@@ -203,6 +203,35 @@ gdn_status gdn_recurrent_step(const void* q, const void* k, const void* v, const
                               int N, int Hk, int Hv, int dk, int dv, void* out, void* stream);
 
 /*
+ * gdn_decode_layer_step -- one decode token of the whole layer core in one launch ([P3] "cache and
+ * state switching": the decode path advances the conv_states cache (the conv's last K-1 inputs)
+ * and the recurrent_states cache (the delta-rule state) by one token; the flowchart's order conv ->
+ * split -> gates -> delta rule -> RMSNormGated(core_attn_out, z); [P2] §2.2 recurrent mode and
+ * §3.2 norm).  Per sequence it equals
+ *     gdn_causal_conv1d_silu on the one new token with conv_state_in as history (q and k heads
+ *     L2-normalised with l2_eps) -> gdn_gates(a, b) -> gdn_recurrent_step -> gdn_gated_rmsnorm(., z)
+ * except that q, k and v stay fp32 between the conv and the delta rule.
+ * mix            : [N, C] dtype, C = 2*Hk*dk + Hv*dv: the new token's [q | k | v] mix before the
+ *                  conv (channel order as gdn_causal_conv1d_silu's).
+ * a, b           : [N, Hv] dtype.   z: [N, Hv, dv] dtype.
+ * conv_w         : [C, K] fp32.  conv_bias: [C] fp32 or NULL.
+ * conv_state_in  : [N, C, K-1] fp32, the previous K-1 inputs of each channel, oldest first.
+ * conv_state_out : [N, C, K-1] fp32, receives them advanced by this token.  Must not overlap
+ *                  conv_state_in (ping-pong two buffers).  Both may be NULL when K = 1.
+ * A_log, dt_bias : [Hv] fp32.   norm_w: [dv] fp32 (zero-centred, used as 1 + w).
+ * state          : [N, Hv, dv, dk] fp32, read and updated IN PLACE.
+ * y              : [N, Hv, dv] dtype, the gated RMSNorm of the core output (must not overlap the
+ *                  inputs).
+ * Supported: dk = dv = 128, 1 <= K <= 8; mix, z, y, state 16-byte aligned.  N = 0 launches nothing.
+ */
+gdn_status gdn_decode_layer_step(const void* mix, const void* a, const void* b, const void* z,
+                                 gdn_dtype dtype, const float* conv_w, const float* conv_bias,
+                                 int K, const float* conv_state_in, float* conv_state_out,
+                                 const float* A_log, const float* dt_bias, const float* norm_w,
+                                 float l2_eps, float norm_eps, float scale, float* state, int N,
+                                 int Hk, int Hv, int dk, int dv, void* y, void* stream);
+
+/*
  * gdn_gated_rmsnorm -- zero-centred RMSNorm gated by z ([P2] §3.2: weight stored zero-centred and
  * used as (1 + w), normalisation in fp32 with rsqrt(mean(x^2) + eps); [P3] output section: the norm
  * of core_attn_out fuses the z gate in, "like SwiGLU").

@@ -147,6 +147,34 @@ def test_recurrent_rejections(lib):
 
 
 @fake_ptr_only_without_gpu
+def test_decode_layer_rejections(lib):
+    f = lib.gdn_decode_layer_step
+    A2 = ctypes.c_void_p(0x20000000)  # a second, distant fake conv-state buffer
+
+    def call(mix=A16, a=A16, b=A16, z=A16, dt=0, w=A16, bias=NUL, K=4, csi=A16, cso=A2,
+             al=A16, db=A16, nw=A16, l2=1e-6, ne=1e-6, scale=0.1, st=A16, N=4, Hk=16, Hv=32,
+             dk=128, dv=128, y=A16):
+        return f(mix, a, b, z, dt, w, bias, K, csi, cso, al, db, nw, l2, ne, scale, st, N, Hk,
+                 Hv, dk, dv, y, STREAM)
+
+    E, U = gdn.GDN_ERR_INVALID_ARG, gdn.GDN_ERR_UNSUPPORTED
+    assert call(dk=64) == U
+    assert call(dv=64) == U
+    assert call(K=9) == U
+    assert call(K=0) == E
+    assert call(Hv=33) == E
+    assert call(dt=7) == E
+    assert call(st=MIS) == E
+    assert call(y=NUL) == E
+    assert call(csi=NUL) == E
+    assert call(cso=A16) == E       # the advanced history may not overlap the old one
+    assert call(K=1, csi=NUL, cso=NUL, N=0) == gdn.GDN_OK
+    assert call(l2=float("nan")) == E
+    assert call(N=-1) == E
+    assert call(N=0) == gdn.GDN_OK
+
+
+@fake_ptr_only_without_gpu
 def test_conv_rejections(lib):
     f = lib.gdn_causal_conv1d_silu
 

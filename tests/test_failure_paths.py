@@ -6,6 +6,8 @@ GDN_ERR_DEVICE_ARG in the workspace status word; the conv bounds every access by
 and the sequence count whatever cu_seqlens holds.  After each such call the same context must
 still run a correct call: a fault that lost the context would show there.
 """
+import os
+
 import numpy as np
 import pytest
 import torch
@@ -90,3 +92,45 @@ def test_conv_bad_cu_seqlens_stays_in_bounds(kind):
                                            return_state=True)
     assert_bf16_rounding_close(y, ref, "conv after bad cu_seqlens")
     assert np.array_equal(s_out.cpu().double().numpy(), s_ref)
+
+
+DEBUG_LIB = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))),
+                         "gated_deltanet_fwd_b200", "libgdn_debug.so")
+
+
+@pytest.mark.parametrize("T,skip", [(600, 3), (2000, 2)])
+def test_chunk_wait_timeout_reports_and_recovers(T, skip):
+    """The failure-test build of the library (every bounded device wait gives up after about a
+    millisecond) withholds one chunk's tiles from the tensor-core prefill, so nothing lands for the
+    waits on that stage: they run out, the kernels record GDN_ERR_TIMEOUT and every CTA leaves with
+    no copy or MMA in flight.  T = 2000 also runs the intra-sequence scan (three phases).  A normal
+    call on the same context afterwards must be correct: nothing was left allocated or hung."""
+    import ctypes
+    assert os.path.exists(DEBUG_LIB), "build the failure-test library: __graft_entry__.build()"
+    prev = gdn._lib
+    gdn._lib = None
+    try:
+        lib = gdn.load(DEBUG_LIB)
+        lib.gdn_debug_set_skip_chunk.argtypes = [ctypes.c_int]
+        lib.gdn_debug_set_skip_chunk.restype = None
+        x = inputs.rule_inputs(B=1, T=T, Hk=1, Hv=2, dk=128, dv=128, seed=T, s0_std=0.02,
+                               a_mean=-6.0)
+        g, beta = oracle_gates_f32(x)
+        args = (x["q"].to(DEV), x["k"].to(DEV), x["v"].to(DEV), g.to(DEV), beta.to(DEV))
+        S0 = x["initial_state"].to(DEV)
+        ws = torch.empty(gdn.workspace_size(1, 1, T, 1, 2, 128, 128, 64), dtype=torch.uint8,
+                         device=DEV)
+        lib.gdn_debug_set_skip_chunk(skip)
+        try:
+            gdn.gdn_chunk_fwd(*args, initial_state=S0, workspace=ws)
+            assert gdn.workspace_status(ws) == gdn.GDN_ERR_TIMEOUT
+        finally:
+            lib.gdn_debug_set_skip_chunk(-1)
+        out, S = gdn.gdn_chunk_fwd(*args, initial_state=S0, workspace=ws)
+        assert gdn.workspace_status(ws) == gdn.GDN_OK
+        o_ref, S_ref = oracle.gated_delta_rule(x["q"], x["k"], x["v"], g, beta, 128 ** -0.5,
+                                               initial_state=x["initial_state"])
+        assert_bf16_close(out, o_ref, "after a timed-out call: out")
+        assert_bf16_close(S, S_ref, "after a timed-out call: state")
+    finally:
+        gdn._lib = prev
