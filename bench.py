@@ -8,7 +8,8 @@ One JSON line on stdout (rank 0).  The headline `value` is prefill tokens/s of t
 d = 128, bf16, chunk 64, per-sequence fp32 initial states, final states returned); one step is
 gdn_gates + gdn_chunk_fwd over that batch.  The same line carries `decode` (256 sequences x 32
 heads of 128 x 128 fp32 state, one step = 64 consecutive gdn_recurrent_step calls, seqs/s) and
-`layer_core` (B = 2 x 16384 tokens: conv + gates + chunk + gated RMSNorm, tokens/s), each with the
+`layer_core` (B = 2 x 16384 tokens: conv, then gates + chunk + gated RMSNorm in one fused call, tokens/s;
+ the four unfused calls timed beside it), each with the
 roofline of its dominant kernel.  Every input is larger than L2, so no flush is needed between
 iterations.
 
@@ -37,10 +38,14 @@ sys.path.insert(0, ROOT)
 from gated_deltanet_fwd_b200 import inputs  # noqa: E402
 
 METRIC = "gated-delta-rule prefill tokens/s (T=32K) & decode seqs/s; % of roofline"
-# Algorithmic work of the chunk form per token per v-head (d = 128, chunk C = 64):
-# 8*C*d (K K^T, Q K^T, the triangular apply, the intra-chunk output) + 6*d^2 (K S^T, Q S^T and the
-# state update) multiply-adds x 2 = 163,840 FLOP.
-CHUNK_FLOP_PER_TOKEN_HEAD = 8 * 64 * 128 + 6 * 128 * 128
+# Algorithmic work of the chunk form per token per v-head (d = 128, chunk C = 64): 2 FLOP per
+# multiply-add x (4*C*d for K K^T, Q K^T, the triangular apply and the intra-chunk output, + 3*d^2
+# for K S^T, Q S^T and the state update) = 163,840 FLOP.
+CHUNK_FLOP_PER_TOKEN_HEAD = 2 * (4 * 64 * 128 + 3 * 128 * 128)
+
+# Kernels one bf16 d = 128 chunk call launches with a workspace of gdn_chunk_fwd_workspace_size():
+# the scan planner, the per-chunk prep, chain phase 1, the state prefix, chain phase 3.
+CHUNK_LAUNCHES = 5
 
 
 # DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of the dominant kernels, from one ncu
@@ -263,7 +268,7 @@ def bench_prefill(dist, gdn, K, W, peaks):
                              traffic=_traffic("gdn_chunk_fwd", T),
                              traffic_unit="bytes per launch", flop_per_launch=flop,
                              peak_source=peaks["source"] + " bf16 burst"),
-               gpu_launches=2 * K)
+               gpu_launches=(1 + CHUNK_LAUNCHES) * K)
 
     # end to end through the public API from pinned host buffers, H2D and D2H inside the region
     host = {k: x[k].pin_memory() for k in ("q", "k", "v", "a", "b", "initial_state")}
@@ -421,34 +426,54 @@ def bench_layer_core(dist, gdn, K, W, peaks):
     cs_out = torch.empty(B, C, w["K"] - 1, device=dev)
     ws = torch.empty(gdn.workspace_size(B, B, T, Hk, Hv, d, d, 64), dtype=torch.uint8, device=dev)
     # q, k, v are views into the conv output [q | k | v] (token stride C): no copies
-    kt = {"conv": KernelTimer(), "chunk": KernelTimer(), "norm": KernelTimer()}
+    kt = {"conv": KernelTimer(), "core": KernelTimer()}
     qv = y[:, :, :Hk * d].view(B, T, Hk, d)
     kv = y[:, :, Hk * d:2 * Hk * d].view(B, T, Hk, d)
     vv = y[:, :, 2 * Hk * d:].view(B, T, Hv, d)
     yout = torch.empty_like(core)
 
+    def conv():
+        gdn.gdn_causal_conv1d_silu(mix, conv_w, None, n_l2norm_ch=2 * Hk * d, l2norm_group=d,
+                                   conv_state_out=cs_out, y=y)
+
+    # the layer core as two calls: conv (+ SiLU + q/k L2 norm), then gates + chunked delta rule +
+    # gated RMSNorm fused into the chunk kernels
     def step(timed):
         run = (lambda name, f: kt[name](f)) if timed else (lambda name, f: f())
-        run("conv", lambda: gdn.gdn_causal_conv1d_silu(mix, conv_w, None, n_l2norm_ch=2 * Hk * d,
-                                                       l2norm_group=d, conv_state_out=cs_out,
-                                                       y=y))
-        gdn.gdn_gates(a, b, A_log, dt_bias, g=g, beta=beta)
+        run("conv", conv)
+        run("core", lambda: gdn.gdn_chunk_fwd_gated_norm(
+            qv, kv, vv, a, b, A_log, dt_bias, z, norm_w, norm_eps=w["eps"], scale=d ** -0.5,
+            y=yout, final_state=S_T, workspace=ws))
+
+    ms = timed_region(dist, step, K, W)
+    status = gdn.workspace_status(ws)
+    if status != 0:
+        raise RuntimeError(f"device status {status} after the fused layer core")
+    per = {k_: t.mean_ms() for k_, t in kt.items()}
+
+    # the same four steps as separate calls, for comparison
+    ku = {"conv": KernelTimer(), "gates": KernelTimer(), "chunk": KernelTimer(),
+          "norm": KernelTimer()}
+
+    def step_unfused(timed):
+        run = (lambda name, f: ku[name](f)) if timed else (lambda name, f: f())
+        run("conv", conv)
+        run("gates", lambda: gdn.gdn_gates(a, b, A_log, dt_bias, g=g, beta=beta))
         run("chunk", lambda: gdn.gdn_chunk_fwd(qv, kv, vv, g, beta, scale=d ** -0.5, chunk=64,
                                                out=core, final_state=S_T, workspace=ws))
         run("norm", lambda: gdn.gdn_gated_rmsnorm(core, z, norm_w, eps=w["eps"], y=yout))
 
-    ms = timed_region(dist, step, K, W)
-    per = {k_: t.mean_ms() for k_, t in kt.items()}
+    ms_u = timed_region(dist, step_unfused, K, W)
+    per_u = {k_: t.mean_ms() for k_, t in ku.items()}
     n_tok = B * T
     conv_bytes = 2 * n_tok * C * 2
-    norm_bytes = 3 * n_tok * Hv * d * 2
     flop = n_tok * Hv * CHUNK_FLOP_PER_TOKEN_HEAD
     return dict(value=n_tok * K * dist.world / (ms * 1e-3), unit="tokens/s", ms_per_step=ms / K,
                 kernels_ms=per,
                 conv_hbm_frac=conv_bytes / (per["conv"] * 1e-3) / 1e9 / peaks["hbm"],
-                norm_hbm_frac=norm_bytes / (per["norm"] * 1e-3) / 1e9 / peaks["hbm"],
-                chunk_tensor_frac=flop / (per["chunk"] * 1e-3) / 1e12 / peaks["bf16"],
-                gpu_launches=4 * K)
+                core_tensor_frac=flop / (per["core"] * 1e-3) / 1e12 / peaks["bf16"],
+                unfused=dict(ms_per_step=ms_u / K, kernels_ms=per_u),
+                gpu_launches=(1 + CHUNK_LAUNCHES) * K)
 
 
 # ------------------------------------------------------------------ CPU oracle --------------

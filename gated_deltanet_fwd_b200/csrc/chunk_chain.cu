@@ -48,7 +48,9 @@ constexpr uint32_t ST_TP = 49152;      // [T'; P]: 128 rows x 128 B
 constexpr uint32_t ST_GD = 65536;      // Gamma[64], d[64] fp32
 constexpr uint32_t STAGE = 66560;      // 65 KB, a multiple of 1024
 constexpr uint32_t SM_GAM = 2 * STAGE;      // Gamma of the two chunks whose outputs are pending
-constexpr uint32_t SM_BAR = SM_GAM + 512;
+constexpr uint32_t SM_ROWS = SM_GAM + 512;   // fused norm: the chunk's outputs, 64 rows x 128 fp32
+constexpr uint32_t SM_Z = SM_ROWS + 32768;   // fused norm: the chunk's z gate, 128 x 128 B
+constexpr uint32_t SM_BAR = SM_Z + 16384;
 constexpr uint32_t SM_USED = SM_BAR + 256;
 constexpr uint32_t CH_SMEM = SM_USED + 1024;
 constexpr uint32_t STAGE_TX = 4 * 16384 + 512;
@@ -58,7 +60,7 @@ static_assert(ST_V == ST_KQ + 32768 && ST_TP == ST_V + 16384, "stage layout");
 enum { B_FULL0 = 0, B_EMPTY0 = 2, B_K = 4, B_U = 5, B_S = 6, B_O = 7, B_DRAIN = 8, B_N = 9 };
 
 // named barriers: producer/consumer hand-offs to the MMA issuer and between the two groups
-enum { NB_X = 1, NB_U = 2, NB_S = 3, NB_SR = 4 };
+enum { NB_X = 1, NB_U = 2, NB_S = 3, NB_SR = 4, NB_H = 5 };
 constexpr int NB_ALL = 288;  // epilogue group + side group + issuer warp
 constexpr int NB_EI = 160;   // epilogue group + issuer warp
 constexpr int NB_EH = 256;   // epilogue group + side group
@@ -98,6 +100,11 @@ struct ChainParams {
   float* st;        // state arrays SOUT, BSEG, MSEG, SIN (scan phases only)
   int debug_skip_chunk;  // failure-test builds only: the producer withholds this chunk's tiles
   unsigned long long* trace;  // phase timing (trace builds only), else unused
+  // fused gated RMSNorm of the outputs (z set): out receives y = o rsqrt(mean o^2 + eps)
+  // (1 + w) silu(z) per (token, head)
+  const __nv_bfloat16* z;
+  const float* norm_w;
+  float norm_eps;
 };
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
@@ -457,23 +464,116 @@ __global__ void __launch_bounds__(CH_THREADS, 1) chunk_chain_kernel(
       if (t4 < 64) gam_o[(c & 1) * 64 + t4] = gd[t4];
       const float gl = gd[63];
 #pragma unroll
-      for (int hh = 0; hh < 2; ++hh) {
-        float v[64];
-        ld64(tmem + lo + TM_S + 64 * hh, v);
+      for (int hh = 0; hh < 4; ++hh) {
+        float v[32];
+        tmem_ld32(tmem + lo + TM_S + 32 * hh, v);
         tmem_ld_wait();
 #pragma unroll
-        for (int q = 0; q < 64; ++q) v[q] *= gl;
+        for (int q = 0; q < 32; ++q) v[q] *= gl;
 #pragma unroll
-        for (int q4 = 0; q4 < 4; ++q4)
-          tmem_st16(tmem + lo + TM_S + 64 * hh + 16 * q4, *reinterpret_cast<float(*)[16]>(v + 16 * q4));
+        for (int q4 = 0; q4 < 2; ++q4)
+          tmem_st16(tmem + lo + TM_S + 32 * hh + 16 * q4, *reinterpret_cast<float(*)[16]>(v + 16 * q4));
       }
       tmem_st_wait();
     };
     named_bar_arrive(NB_S, NB_ALL);  // D_q is free
     scale_s(0);
     tc_fence_before();
+    // fused norm: thread t4 owns half `half` of token row r of each chunk; its 128 bytes of z are
+    // copied into its own slot of SM_Z at the top of the chunk (the 16-byte pieces in an order
+    // rotated by t4, so that eight neighbouring threads hit eight different bank groups)
+    unsigned char* zs = smem + SM_Z + t4 * 128;
+    const int zr_row = t4 >> 1, zr_half = t4 & 1;
     for (int c = 0; c < nchunks; ++c) {
+      if (P.z && has_out) {
+        const int64_t t0 = chunk_t0(c);
+        if (zr_row < (int)min((int64_t)tm::C, s_end - t0)) {
+          const __nv_bfloat16* zrow =
+              P.z + ((size_t)(t0 + zr_row) * P.Hv + h) * tm::D + 64 * zr_half;
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const int cc = (i + t4) & 7;
+            cp_async16(zs + 16 * cc, zrow + 8 * cc);
+          }
+        }
+      }
       named_bar(NB_U, NB_ALL);  // S scaled by Gamma_63(c); a full barrier (see the other group)
+      if (P.z) {
+        // ---- outputs of chunk c with the gated RMSNorm: O^T = diag(Gamma) (S Q^T) + U^T P^T is
+        // staged as [row][column] fp32, then each thread takes half of a token row: its sum of
+        // squares (with the other half's), the z gate and the norm weight, and 64 bytes of y
+        float* rows = reinterpret_cast<float*>(smem + SM_ROWS);
+        named_bar(NB_H, 128);  // the previous chunk's rows have been read
+        const bool o_ok = has_out && wait(B_O, c & 1);
+        if (t4 == 0) CH_TS(c, 12);
+        if (o_ok) {
+          tc_fence_after();
+          const float* gm = gam_o + (c & 1) * 64;
+          float* col = rows + j;
+#pragma unroll 1
+          for (int q16 = 0; q16 < 4; ++q16) {
+            float dq[16], doo[16];
+            tmem_ld16(tmem + lo + TM_Q + 16 * q16, dq);
+            tmem_ld16(tmem + lo + TM_K + 16 * q16, doo);
+            tmem_ld_wait();
+#pragma unroll
+            for (int q = 0; q < 16; ++q)
+              col[(16 * q16 + q) * 128] = P.scale * fmaf(gm[16 * q16 + q], dq[q], doo[q]);
+          }
+        }
+        tc_fence_before();
+        if (c + 1 < nchunks) named_bar_arrive(NB_S, NB_ALL);  // D_q and D_o read
+        named_bar(NB_H, 128);  // the chunk's rows are complete
+        // ---- S scaled by Gamma_63 for chunk c + 1 (needed before the issuer's next NB_U)
+        if (c + 1 < nchunks) {
+          scale_s(c + 1);
+          if (t4 == 0) CH_TS(c, 14);
+          tc_fence_before();
+        }
+        cp_async_wait_all();  // this thread's z pieces of chunk c
+        if (o_ok && !*abort_flag) {
+          const int64_t t0 = chunk_t0(c);
+          const int L = (int)min((int64_t)tm::C, s_end - t0);
+          const int r = zr_row, half = zr_half;
+          // float4 q of the half row, read in an order rotated by t4 (bank groups as for z)
+          const float4* xr = reinterpret_cast<const float4*>(rows + r * 128 + 64 * half);
+          float ssq = 0.0f;
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const float4 x = xr[(i + t4) & 15];
+            ssq = fmaf(x.x, x.x, fmaf(x.y, x.y, fmaf(x.z, x.z, fmaf(x.w, x.w, ssq))));
+          }
+          ssq += __shfl_xor_sync(0xffffffffu, ssq, 1);
+          const float inv = rsqrtf(ssq * (1.0f / tm::D) + P.norm_eps);
+          if (r < L) {
+            const size_t off = ((size_t)(t0 + r) * P.Hv + h) * tm::D + 64 * half;
+            uint4* yr = reinterpret_cast<uint4*>(P.out + off);
+            const float* wh = P.norm_w + 64 * half;
+#pragma unroll 1
+            for (int i = 0; i < 8; ++i) {
+              const int cc = (i + t4) & 7;
+              const uint4 zu = *reinterpret_cast<const uint4*>(zs + 16 * cc);
+              const uint32_t zw[4] = {zu.x, zu.y, zu.z, zu.w};
+              const float4 x0 = xr[2 * cc], x1 = xr[2 * cc + 1];
+              const float xv[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+              const float4 w0 = __ldg(reinterpret_cast<const float4*>(wh + 8 * cc));
+              const float4 w1 = __ldg(reinterpret_cast<const float4*>(wh + 8 * cc + 4));
+              const float wv[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+              uint32_t pk[4];
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const float2 zz = make_float2(__uint_as_float(zw[e] << 16),
+                                              __uint_as_float(zw[e] & 0xffff0000u));
+                pk[e] = pack_bf16x2(xv[2 * e] * inv * (1.0f + wv[2 * e]) * siluf_(zz.x),
+                                    xv[2 * e + 1] * inv * (1.0f + wv[2 * e + 1]) * siluf_(zz.y));
+              }
+              yr[cc] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+            }
+          }
+        }
+        if (t4 == 0) CH_TS(c, 13);
+        continue;
+      }
       // ---- outputs of chunk c: O^T = diag(Gamma) (S Q^T) + U^T P^T, held as scaled bf16 pairs
       // (rows 2q, 2q + 1) of value column j
       uint32_t ob[32];
@@ -565,7 +665,8 @@ unsigned long long* g_chain_trace = nullptr;  // trace builds: device buffer of 
 cudaError_t launch_chunk_chain(const void* q, const void* k, const void* v, TokStrides ts,
                                float scale, const float* S0, const int32_t* cu, int N, int B,
                                int64_t T, int Hk, int Hv, void* out, float* S_T, void* ws,
-                               int phase, int64_t lseg, int* status, cudaStream_t s) {
+                               int phase, int64_t lseg, int* status, cudaStream_t s,
+                               const ChunkFusion& fuse) {
   const int64_t n_tok = (int64_t)B * T;
   const int64_t msegs = tm::max_segs(N, n_tok, lseg);  // lseg: the smallest the planner may pick
   // units per v-head: phase 0 one per sequence; phase 1 at most one per sequence and two per
@@ -601,6 +702,9 @@ cudaError_t launch_chunk_chain(const void* q, const void* k, const void* v, TokS
                     : reinterpret_cast<float*>(wsb + tm::states_offset(N, n_tok, Hv));
   p.debug_skip_chunk = g_debug_skip_chunk;
   p.trace = g_chain_trace;
+  p.z = fuse.z;
+  p.norm_w = fuse.norm_w;
+  p.norm_eps = fuse.norm_eps;
   static bool attr_set = false;  // idempotent attribute; a benign race between host threads
   if (!attr_set) {
     cudaError_t e = cudaFuncSetAttribute(chunk_chain_kernel,

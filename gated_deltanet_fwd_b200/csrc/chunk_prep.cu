@@ -73,6 +73,11 @@ struct PrepParams {
   int64_t gd_off;  // byte offset of the GD array
   int N, Hk, Hv;
   unsigned long long* trace;  // phase timing (trace builds only), else unused
+  // fused gates: g and beta computed here from a, b (bf16) when a is set
+  const __nv_bfloat16* a;
+  const __nv_bfloat16* b;
+  const float* A_log;
+  const float* dt_bias;
 };
 
 __device__ __forceinline__ float ex2f(float x) {
@@ -282,13 +287,26 @@ __global__ void __launch_bounds__(PP_THREADS, 2) chunk_prep_kernel(const PrepPar
       const int h = hk * G + h0 + warp;
       float* gl2 = gl2_all + warp * 128;
       float x0 = 0.f, x1 = 0.f, b0 = 0.f, b1 = 0.f;
-      if (lane < L) {
-        x0 = gxp[(t0 + lane) * P.Hv + h];
-        b0 = bxp[(t0 + lane) * P.Hv + h];
-      }
-      if (32 + lane < L) {
-        x1 = gxp[(t0 + 32 + lane) * P.Hv + h];
-        b1 = bxp[(t0 + 32 + lane) * P.Hv + h];
+      if (P.a) {
+        // the gates of the layer: beta = sigmoid(b), g = -exp(A_log) softplus(a + dt_bias)
+        const float ea = expf(__ldg(P.A_log + h)), db = __ldg(P.dt_bias + h);
+        if (lane < L) {
+          x0 = -ea * softplusf_(__bfloat162float(P.a[(t0 + lane) * P.Hv + h]) + db);
+          b0 = sigmoidf_(__bfloat162float(P.b[(t0 + lane) * P.Hv + h]));
+        }
+        if (32 + lane < L) {
+          x1 = -ea * softplusf_(__bfloat162float(P.a[(t0 + 32 + lane) * P.Hv + h]) + db);
+          b1 = sigmoidf_(__bfloat162float(P.b[(t0 + 32 + lane) * P.Hv + h]));
+        }
+      } else {
+        if (lane < L) {
+          x0 = gxp[(t0 + lane) * P.Hv + h];
+          b0 = bxp[(t0 + lane) * P.Hv + h];
+        }
+        if (32 + lane < L) {
+          x1 = gxp[(t0 + 32 + lane) * P.Hv + h];
+          b1 = bxp[(t0 + 32 + lane) * P.Hv + h];
+        }
       }
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
@@ -410,7 +428,8 @@ unsigned long long* g_prep_trace = nullptr;  // trace builds: device buffer of 8
 
 cudaError_t launch_chunk_prep(const void* q, const void* k, TokStrides ts, const float* g,
                               const float* beta, const int32_t* cu, int N, int B, int64_t T,
-                              int Hk, int Hv, void* ws, int* status, cudaStream_t s) {
+                              int Hk, int Hv, void* ws, int* status, cudaStream_t s,
+                              const ChunkFusion& fuse) {
   const int64_t n_tok = (int64_t)B * T;
   const int64_t slots = tm::max_slots(N, n_tok);
   if (slots <= 0 || n_tok == 0) return cudaSuccess;
@@ -431,6 +450,10 @@ cudaError_t launch_chunk_prep(const void* q, const void* k, TokStrides ts, const
   p.Hk = Hk;
   p.Hv = Hv;
   p.trace = g_prep_trace;
+  p.a = fuse.a;
+  p.b = fuse.b;
+  p.A_log = fuse.A_log;
+  p.dt_bias = fuse.dt_bias;
   static bool attr_set = false;  // idempotent attribute; a benign race between host threads
   if (!attr_set) {
     cudaError_t e = cudaFuncSetAttribute(chunk_prep_kernel,

@@ -31,6 +31,47 @@ int sm_count() {
     return 148;
   return sms;
 }
+// The two-kernel tensor-core prefill (bf16, dk = dv = 128, chunk 64) when the workspace has room
+// for it: with room for the scan's states the planner picks a segment length (or none) and the
+// call runs prep, phase 1, prefix, phase 3; with room only for the per-chunk operands, prep and one
+// chain per (sequence, v-head).  Returns false (nothing launched) when the workspace is too small.
+bool run_two_kernel(const void* q, const void* k, const void* v, TokStrides ts, const float* g,
+                    const float* beta, float scale, const float* S0, const int32_t* cu, int N,
+                    int B, int64_t T, int Hk, int Hv, void* out, float* S_T, void* ws,
+                    size_t ws_bytes, int* status, cudaStream_t s, const ChunkFusion& fuse,
+                    cudaError_t* err) {
+  const int64_t n_tok = (int64_t)B * T;
+  const int sms = sm_count();
+  const int64_t lseg = gdn::tm::scan_segment_tokens(n_tok, Hv, sms);
+  cudaError_t e;
+  if (lseg > 0 && ws_bytes >= gdn::tm::workspace_bytes_scan(N, n_tok, Hv, lseg)) {
+    e = launch_scan_plan(cu, N, B, T, Hv, sms, lseg, ws, status, s);
+    if (e == cudaSuccess)
+      e = launch_chunk_prep(q, k, ts, g, beta, cu, N, B, T, Hk, Hv, ws, status, s, fuse);
+    if (e == cudaSuccess)
+      e = launch_chunk_chain(q, k, v, ts, scale, S0, cu, N, B, T, Hk, Hv, out, S_T, ws, 1, lseg,
+                             status, s, fuse);
+    if (e == cudaSuccess) e = launch_scan_prefix(cu, N, B, T, Hv, lseg, ws, status, s);
+    if (e == cudaSuccess)
+      e = launch_chunk_chain(q, k, v, ts, scale, S0, cu, N, B, T, Hk, Hv, out, S_T, ws, 3, lseg,
+                             status, s, fuse);
+  } else if (ws_bytes >= gdn::tm::workspace_bytes(N, n_tok, Hv)) {
+    e = launch_chunk_prep(q, k, ts, g, beta, cu, N, B, T, Hk, Hv, ws, status, s, fuse);
+    if (e == cudaSuccess)
+      e = launch_chunk_chain(q, k, v, ts, scale, S0, cu, N, B, T, Hk, Hv, out, S_T, ws, 0, 0,
+                             status, s, fuse);
+  } else {
+    return false;
+  }
+  *err = e;
+  return true;
+}
+
+inline bool overlaps(const void* x, size_t xb, const void* y, size_t yb) {
+  const char* a = (const char*)x;
+  const char* b = (const char*)y;
+  return a < b + yb && b < a + xb;
+}
 
 }  // namespace
 
@@ -170,32 +211,9 @@ gdn_status gdn_chunk_fwd_strided(const void* q, int64_t q_tok_stride, const void
   const TokStrides ts{q_tok_stride, k_tok_stride, v_tok_stride};
   cudaError_t e;
   if (dtype == GDN_BF16 && dk == gdn::tm::D && dv == gdn::tm::D && chunk == gdn::tm::C) {
-    const int64_t n_tok = (int64_t)B * T;
-    const int sms = sm_count();
-    const int64_t lseg = gdn::tm::scan_segment_tokens(n_tok, Hv, sms);
-    if (lseg > 0 && workspace_bytes >= gdn::tm::workspace_bytes_scan(N, n_tok, Hv, lseg)) {
-      // the planner picks the segment length (or none); prep over all (chunk, k-head); chains of
-      // segment 0 and the middle segments' maps; the prefix over segments; chains of the later
-      // segments from their entry states
-      e = launch_scan_plan(cu_seqlens, N, B, T, Hv, sms, lseg, workspace, status, s);
-      if (e == cudaSuccess)
-        e = launch_chunk_prep(q, k, ts, g, beta, cu_seqlens, N, B, T, Hk, Hv, workspace, status,
-                              s);
-      if (e == cudaSuccess)
-        e = launch_chunk_chain(q, k, v, ts, scale, initial_state, cu_seqlens, N, B, T, Hk, Hv,
-                               out, final_state, workspace, 1, lseg, status, s);
-      if (e == cudaSuccess)
-        e = launch_scan_prefix(cu_seqlens, N, B, T, Hv, lseg, workspace, status, s);
-      if (e == cudaSuccess)
-        e = launch_chunk_chain(q, k, v, ts, scale, initial_state, cu_seqlens, N, B, T, Hk, Hv,
-                               out, final_state, workspace, 3, lseg, status, s);
-    } else if (workspace_bytes >= gdn::tm::workspace_bytes(N, n_tok, Hv)) {
-      // prep over all (chunk, k-head), then one chain per (sequence, v-head)
-      e = launch_chunk_prep(q, k, ts, g, beta, cu_seqlens, N, B, T, Hk, Hv, workspace, status, s);
-      if (e == cudaSuccess)
-        e = launch_chunk_chain(q, k, v, ts, scale, initial_state, cu_seqlens, N, B, T, Hk, Hv,
-                               out, final_state, workspace, 0, 0, status, s);
-    } else {
+    if (!run_two_kernel(q, k, v, ts, g, beta, scale, initial_state, cu_seqlens, N, B, T, Hk, Hv,
+                        out, final_state, workspace, workspace_bytes, status, s, ChunkFusion(),
+                        &e)) {
       e = launch_chunk_tc(q, k, v, ts, g, beta, scale, initial_state, cu_seqlens, N, B, T, Hk,
                           Hv, out, final_state, status, s);
     }
@@ -214,6 +232,63 @@ gdn_status gdn_chunk_fwd(const void* q, const void* k, const void* v, const floa
   return gdn_chunk_fwd_strided(q, (int64_t)Hk * dk, k, (int64_t)Hk * dk, v, (int64_t)Hv * dv, g,
                                beta, dtype, scale, initial_state, cu_seqlens, N, B, T, Hk, Hv, dk,
                                dv, chunk, out, final_state, workspace, workspace_bytes, stream);
+}
+
+gdn_status gdn_chunk_fwd_gated_norm(const void* q, int64_t q_tok_stride, const void* k,
+                                    int64_t k_tok_stride, const void* v, int64_t v_tok_stride,
+                                    const void* a, const void* b, const float* A_log,
+                                    const float* dt_bias, const void* z, const float* norm_w,
+                                    float norm_eps, gdn_dtype dtype, float scale,
+                                    const float* initial_state, const int32_t* cu_seqlens, int N,
+                                    int B, int64_t T, int Hk, int Hv, int dk, int dv, int chunk,
+                                    void* y, float* final_state, void* workspace,
+                                    size_t workspace_bytes, void* stream) {
+  if (bad_dtype(dtype) || N < 0 || B < 0 || T < 0 || Hk < 1 || Hv < 1 || dk < 1 || dv < 1)
+    return GDN_ERR_INVALID_ARG;
+  if (Hv % Hk != 0) return GDN_ERR_INVALID_ARG;
+  if (cu_seqlens ? (B != 1) : (N != B)) return GDN_ERR_INVALID_ARG;
+  if (!(scale == scale) || !(norm_eps >= 0.0f)) return GDN_ERR_INVALID_ARG;
+  if (q_tok_stride < (int64_t)Hk * dk || k_tok_stride < (int64_t)Hk * dk ||
+      v_tok_stride < (int64_t)Hv * dv || q_tok_stride % 8 || k_tok_stride % 8 ||
+      v_tok_stride % 8)
+    return GDN_ERR_INVALID_ARG;
+  if (!workspace || workspace_bytes < kStatusBytes) return GDN_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return GDN_ERR_INVALID_ARG;
+  if (dtype != GDN_BF16 || dk != gdn::tm::D || dv != gdn::tm::D || chunk != gdn::tm::C)
+    return GDN_ERR_UNSUPPORTED;
+  const int64_t n_tok = (int64_t)B * T;
+  if (workspace_bytes < gdn::tm::workspace_bytes(N, n_tok, Hv)) return GDN_ERR_UNSUPPORTED;
+  if (N == 0) return GDN_OK;
+  if (n_tok > 0) {
+    if (!ptr_ok(q) || !ptr_ok(k) || !ptr_ok(v) || !ptr_ok(z) || !ptr_ok(y) || !ptr_ok(norm_w))
+      return GDN_ERR_INVALID_ARG;
+    if (!a || !b || !A_log || !dt_bias) return GDN_ERR_INVALID_ARG;
+    const size_t zb = (size_t)n_tok * Hv * dv * 2;
+    if (overlaps(y, zb, z, zb)) return GDN_ERR_INVALID_ARG;
+  }
+  if ((initial_state && !aligned16(initial_state)) || (final_state && !aligned16(final_state)))
+    return GDN_ERR_INVALID_ARG;
+  if (cu_seqlens && ((uintptr_t)cu_seqlens & 3u)) return GDN_ERR_INVALID_ARG;
+  if (initial_state && final_state) {
+    const size_t bytes = (size_t)N * Hv * dv * dk * sizeof(float);
+    if (overlaps(initial_state, bytes, final_state, bytes)) return GDN_ERR_INVALID_ARG;
+  }
+  cudaStream_t s = as_stream(stream);
+  int* status = reinterpret_cast<int*>(workspace);
+  if (cudaMemsetAsync(status, 0, sizeof(int), s) != cudaSuccess) return GDN_ERR_CUDA;
+  ChunkFusion fuse;
+  fuse.a = reinterpret_cast<const __nv_bfloat16*>(a);
+  fuse.b = reinterpret_cast<const __nv_bfloat16*>(b);
+  fuse.A_log = A_log;
+  fuse.dt_bias = dt_bias;
+  fuse.z = reinterpret_cast<const __nv_bfloat16*>(z);
+  fuse.norm_w = norm_w;
+  fuse.norm_eps = norm_eps;
+  const TokStrides ts{q_tok_stride, k_tok_stride, v_tok_stride};
+  cudaError_t e = cudaSuccess;
+  run_two_kernel(q, k, v, ts, nullptr, nullptr, scale, initial_state, cu_seqlens, N, B, T, Hk,
+                 Hv, y, final_state, workspace, workspace_bytes, status, s, fuse, &e);
+  return from_cuda(e);
 }
 
 gdn_status gdn_recurrent_step(const void* q, const void* k, const void* v, const float* g,

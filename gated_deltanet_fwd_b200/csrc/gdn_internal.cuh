@@ -170,6 +170,19 @@ cudaError_t launch_chunk_simt(const void* q, const void* k, const void* v, TokSt
                               int dv, int chunk, void* out, float* S_T, int* status,
                               cudaStream_t s);
 
+// Optional fusions of the layer's neighbouring steps into the two-kernel tensor-core prefill: the
+// gates computed from their pre-activations inside the prep kernel (a, b set), and the gated
+// RMSNorm applied to the outputs in the chain's output epilogue (z set; `out` then receives y).
+struct ChunkFusion {
+  const __nv_bfloat16* a = nullptr;  // [tokens, Hv] gate pre-activations (fused gates when set)
+  const __nv_bfloat16* b = nullptr;
+  const float* A_log = nullptr;
+  const float* dt_bias = nullptr;
+  const __nv_bfloat16* z = nullptr;  // [tokens, Hv, dv] (fused gated RMSNorm when set)
+  const float* norm_w = nullptr;
+  float norm_eps = 0.0f;
+};
+
 // TMA tensor maps (tma_maps.cu), 128-byte swizzle, bf16:
 //   make_tok_map:    [rows, heads, 128] with `tok_stride` elements between rows; box {64, 1, 64}
 //   make_rows64_map: [rows, 64] dense;                                          box {64, box_rows}
@@ -180,14 +193,16 @@ bool make_rows64_map(CUtensorMap* m, const void* base, int64_t rows, uint32_t bo
 // then the chain kernel.  `ws` holds at least tm::workspace_bytes(N, B*T, Hv) bytes.
 cudaError_t launch_chunk_prep(const void* q, const void* k, TokStrides ts, const float* g,
                               const float* beta, const int32_t* cu, int N, int B, int64_t T,
-                              int Hk, int Hv, void* ws, int* status, cudaStream_t s);
+                              int Hk, int Hv, void* ws, int* status, cudaStream_t s,
+                              const ChunkFusion& fuse = ChunkFusion());
 // phase 0: one chain per (sequence, v-head); phases 1 and 3 (with launch_scan_prefix between
 // them): the intra-sequence scan with segments of lseg tokens (chunk_tm.cuh), for which `ws` holds
 // at least tm::workspace_bytes_scan(N, B*T, Hv, lseg) bytes.
 cudaError_t launch_chunk_chain(const void* q, const void* k, const void* v, TokStrides ts,
                                float scale, const float* S0, const int32_t* cu, int N, int B,
                                int64_t T, int Hk, int Hv, void* out, float* S_T, void* ws,
-                               int phase, int64_t lseg, int* status, cudaStream_t s);
+                               int phase, int64_t lseg, int* status, cudaStream_t s,
+                               const ChunkFusion& fuse = ChunkFusion());
 // One-thread planner: writes the call's segment length (0, lseg, 2 lseg or 4 lseg) into the
 // workspace for the two chain phases and the prefix to read.
 cudaError_t launch_scan_plan(const int32_t* cu, int N, int B, int64_t T, int Hv, int sms,

@@ -34,6 +34,9 @@ SIGNATURES = {
                            _P, _P, _P, _SZ, _P]),
     "gdn_chunk_fwd_strided": (_I, [_P, _I64, _P, _I64, _P, _I64, _P, _P, _I, _F, _P, _P, _I, _I,
                                    _I64, _I, _I, _I, _I, _I, _P, _P, _P, _SZ, _P]),
+    "gdn_chunk_fwd_gated_norm": (_I, [_P, _I64, _P, _I64, _P, _I64, _P, _P, _P, _P, _P, _P, _F,
+                                      _I, _F, _P, _P, _I, _I, _I64, _I, _I, _I, _I, _I, _P, _P,
+                                      _P, _SZ, _P]),
     "gdn_chunk_fwd_noalloc": (_I, [_P, _P, _P, _P, _P, _I, _F, _P, _P, _I, _I, _I64, _I, _I, _I,
                                    _I, _I, _P, _P, _P]),
     "gdn_chunk_fwd_workspace_size": (_SZ, [_I, _I, _I64, _I, _I, _I, _I, _I]),
@@ -187,6 +190,36 @@ def gdn_chunk_fwd(q, k, v, g, beta, scale=None, initial_state=None, cu_seqlens=N
             _ptr(initial_state), _ptr(cu_seqlens), N, B, T, Hk, Hv, dk, dv, chunk, _ptr(out),
             _ptr(final_state), _ptr(workspace), ws_b, _stream(q)))
     return out, final_state
+
+
+def gdn_chunk_fwd_gated_norm(q, k, v, a, b, A_log, dt_bias, z, norm_w, norm_eps=1e-6, scale=None,
+                             initial_state=None, cu_seqlens=None, y=None, final_state=None,
+                             output_final_state=True, workspace=None):
+    """Layer core after the conv in one call: gates(a, b) -> chunked delta rule -> gated RMSNorm
+    with z.  q, k: [B, T, Hk, 128]; v: [B, T, Hv, 128] (may be strided views of the conv output);
+    a, b: [B, T, Hv] bf16; z: [B, T, Hv, 128] bf16.  Returns (y, final_state)."""
+    _cuda(a, b, A_log, dt_bias, z, norm_w, initial_state, cu_seqlens, y, final_state, workspace)
+    if len({t.dtype for t in (q, k, v, a, b, z)}) != 1:
+        raise TypeError("q, k, v, a, b and z must share one activation dtype")
+    qs, ks, vs = _tok_stride(q), _tok_stride(k), _tok_stride(v)
+    if qs is None or ks is None or vs is None:
+        raise ValueError("q, k, v must be CUDA [B, T, H, d] tensors with each token's heads packed")
+    B, T, Hk, dk = q.shape
+    Hv, dv = v.shape[2], v.shape[3]
+    N = cu_seqlens.numel() - 1 if cu_seqlens is not None else B
+    scale = dk ** -0.5 if scale is None else scale
+    y = torch.empty(v.shape, dtype=v.dtype, device=v.device) if y is None else y
+    if final_state is None and output_final_state:
+        final_state = torch.empty((N, Hv, dv, dk), dtype=torch.float32, device=q.device)
+    if workspace is None:
+        workspace = torch.empty(workspace_size(N, B, T, Hk, Hv, dk, dv, 64), dtype=torch.uint8,
+                                device=q.device)
+    _check("gdn_chunk_fwd_gated_norm", load().gdn_chunk_fwd_gated_norm(
+        _ptr(q), qs, _ptr(k), ks, _ptr(v), vs, _ptr(a), _ptr(b), _ptr(A_log), _ptr(dt_bias),
+        _ptr(z), _ptr(norm_w), float(norm_eps), _dt(q), float(scale), _ptr(initial_state),
+        _ptr(cu_seqlens), N, B, T, Hk, Hv, dk, dv, 64, _ptr(y), _ptr(final_state),
+        _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(q)))
+    return y, final_state
 
 
 def gdn_recurrent_step(q, k, v, g, beta, state, scale=None, out=None):

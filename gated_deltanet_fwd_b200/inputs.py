@@ -169,3 +169,19 @@ def layer_core_inputs(*, B, T, Hk, Hv, dk, dv, K=4, dtype="bf16", seed=0, seqlen
     cu = cu_from_lengths(seqlens) if seqlens is not None else None
     return dict(mix=mix, z=z, a=a, b=b, A_log=A_log, dt_bias=dt_bias, conv_w=conv_w,
                 norm_w=norm_w, cu_seqlens=cu, C=C)
+
+
+def fused_core_inputs(*, B, T, Hk, Hv, dk, dv, seed=0, seqlens=None, s0_std=None, a_mean=0.0,
+                      **_unused):
+    """Inputs of the layer core after the conv (q, k, v already L2-normalised as the conv leaves
+    them): rule_inputs' q, k, v, initial state and cu_seqlens in bf16, with a, b rounded to bf16
+    (they come out of a bf16 projection), z [B,T,Hv,dv] bf16 ~ N(0, 1) and norm_w [dv] fp32
+    ~ N(0, 0.02)."""
+    x = rule_inputs(B=B, T=T, Hk=Hk, Hv=Hv, dk=dk, dv=dv, dtype="bf16", seed=seed,
+                    seqlens=seqlens, s0_std=s0_std, a_mean=a_mean)
+    gen = _gen(seed + 7919)
+    x["a"] = x["a"].to(torch.bfloat16)
+    x["b"] = x["b"].to(torch.bfloat16)
+    x["z"] = _randn(gen, (B, T, Hv, dv)).to(torch.bfloat16)
+    x["norm_w"] = _randn(gen, (dv,), std=0.02)
+    return x

@@ -149,6 +149,37 @@ gdn_status gdn_chunk_fwd_strided(const void* q, int64_t q_tok_stride, const void
                                  size_t workspace_bytes, void* stream);
 
 /*
+ * gdn_chunk_fwd_gated_norm -- the layer core after the conv in one call: the gates, the chunked
+ * gated delta rule and the gated RMSNorm of its output, as in [P3]'s flowchart (split -> gates ->
+ * delta rule -> RMSNormGated(core_attn_out, z)) and [P2] §3.2.  Results equal
+ *     gdn_gates(a, b) -> gdn_chunk_fwd_strided(q, k, v, g, beta) -> gdn_gated_rmsnorm(., z)
+ * except that g, beta and the delta-rule output o are never written to memory: the gates are
+ * computed where the per-chunk operands are prepared, and the norm is applied to the fp32 o before
+ * it is rounded to bf16 (the unfused composition normalises the bf16-rounded o).
+ * q, k, v, strides, scale, initial_state, cu_seqlens, N, B, T, Hk, Hv, final_state, workspace:
+ *                  as gdn_chunk_fwd_strided.
+ * a, b           : [B*T, Hv] bf16 gate pre-activations (as gdn_gates).
+ * A_log, dt_bias : [Hv] fp32 (as gdn_gates).
+ * z              : [B*T, Hv, dv] bf16, the output gate.   norm_w: [dv] fp32 (used as 1 + w).
+ * y              : [B*T, Hv, dv] bf16, the gated RMSNorm of the delta-rule output.  Must not
+ *                  overlap z, q, k or v.
+ * Supported: bf16, dk = dv = 128, chunk = 64, with a workspace of gdn_chunk_fwd_workspace_size()
+ * bytes (one too small for the intra-sequence scan's state arrays but holding the per-chunk
+ * operands runs without the scan); anything else returns GDN_ERR_UNSUPPORTED -- use the three
+ * unfused calls there.  z, y, norm_w 16-byte
+ * aligned.  Device-detected faults land in the workspace status word as for gdn_chunk_fwd.
+ */
+gdn_status gdn_chunk_fwd_gated_norm(const void* q, int64_t q_tok_stride, const void* k,
+                                    int64_t k_tok_stride, const void* v, int64_t v_tok_stride,
+                                    const void* a, const void* b, const float* A_log,
+                                    const float* dt_bias, const void* z, const float* norm_w,
+                                    float norm_eps, gdn_dtype dtype, float scale,
+                                    const float* initial_state, const int32_t* cu_seqlens, int N,
+                                    int B, int64_t T, int Hk, int Hv, int dk, int dv, int chunk,
+                                    void* y, float* final_state, void* workspace,
+                                    size_t workspace_bytes, void* stream);
+
+/*
  * gdn_chunk_fwd_noalloc -- gdn_chunk_fwd for callers that cannot allocate device memory.  The
  * pages have no counterpart: this is a library convenience.
  * Who needs it: code that receives device pointers from another runtime and may not allocate

@@ -128,6 +128,41 @@ def test_chunk_strided_rejections(lib):
 
 
 @fake_ptr_only_without_gpu
+def test_chunk_gated_norm_rejections(lib):
+    f = lib.gdn_chunk_fwd_gated_norm
+    full = 1024 + (1 + 1) * 32 * (16384 + 512)  # per-chunk operands of one 64-token sequence
+
+    Y = P(0x7f0000100000)  # past z's 512 KB
+
+    def call(q=A16, a=A16, b=A16, z=A16, w=A16, y=Y, eps=1e-6, dt=0, s0=NUL, sT=A16, cu=NUL,
+             N=1, B=1, T=64, Hk=16, Hv=32, dk=128, dv=128, chunk=64, ws=A16, wsb=full,
+             qs=2048):
+        return f(q, qs, A16, 2048, A16, 4096, a, b, A16, A16, z, w, eps, dt, 0.1, s0, cu, N, B,
+                 T, Hk, Hv, dk, dv, chunk, y, sT, ws, wsb, STREAM)
+
+    E, U = gdn.GDN_ERR_INVALID_ARG, gdn.GDN_ERR_UNSUPPORTED
+    assert call(dt=1) == U               # fp32 activations: use the unfused calls
+    assert call(dk=64) == U
+    assert call(chunk=32) == U
+    assert call(wsb=4096) == U           # no room for the per-chunk operands
+    assert call(dt=7) == E
+    assert call(Hv=24) == E
+    assert call(eps=-1.0) == E
+    assert call(eps=float("nan")) == E
+    assert call(qs=2047) == E
+    assert call(ws=NUL) == E
+    assert call(a=NUL) == E
+    assert call(b=NUL) == E
+    assert call(z=MIS) == E
+    assert call(w=MIS) == E
+    assert call(y=NUL) == E
+    assert call(z=A16, y=A16) == E       # y overlaps z
+    assert call(s0=A16, sT=A16) == E
+    assert call(N=2, B=1) == E
+    assert call(N=0, B=0) == gdn.GDN_OK
+
+
+@fake_ptr_only_without_gpu
 def test_recurrent_rejections(lib):
     f = lib.gdn_recurrent_step
 

@@ -49,10 +49,16 @@ def test_layer_core_end_to_end_full_size():
     vv = y[:, :, 2 * Hk * d:].view(B, T, Hv, d)
     core, S_T = gdn.gdn_chunk_fwd(qv, kv, vv, g, beta, scale=scale, chunk=64)
     yn = gdn.gdn_gated_rmsnorm(core, x["z"].to(DEV), x["norm_w"].to(DEV), eps=w["eps"])
+    # the same after the conv as one call (gates and norm fused into the chunk kernels)
+    yf, Sf = gdn.gdn_chunk_fwd_gated_norm(qv, kv, vv, x["a"].to(DEV), x["b"].to(DEV),
+                                          x["A_log"].to(DEV), x["dt_bias"].to(DEV),
+                                          x["z"].to(DEV), x["norm_w"].to(DEV), norm_eps=w["eps"],
+                                          scale=scale)
     torch.cuda.synchronize()
     y_gpu, cs_gpu = y.cpu(), cs_out.cpu()
     core_gpu, S_gpu, yn_gpu = core.cpu(), S_T.cpu(), yn.cpu()
-    del mix, y, qv, kv, vv, core, S_T, yn
+    yf_gpu, Sf_gpu = yf.cpu(), Sf.cpu()
+    del mix, y, qv, kv, vv, core, S_T, yn, yf, Sf
 
     # ---- oracle composition in fp64 (one batch row at a time keeps host memory bounded)
     g_ref, b_ref = oracle.gates(x["a"], x["b"], x["A_log"], x["dt_bias"])
@@ -82,3 +88,9 @@ def test_layer_core_end_to_end_full_size():
         record_margin(f"layer core normed output, row {bi}", rel_l2=r, rel_l2_tol=BF16_REL_L2,
                       max_abs=max_abs(yn_gpu[bi:bi + 1], yn_ref))
         assert r <= BF16_REL_L2
+        # the fused call: same bound on its normed output and final state
+        rf = rel_l2(yf_gpu[bi:bi + 1], yn_ref)
+        record_margin(f"layer core fused normed output, row {bi}", rel_l2=rf,
+                      rel_l2_tol=BF16_REL_L2, max_abs=max_abs(yf_gpu[bi:bi + 1], yn_ref))
+        assert rf <= BF16_REL_L2
+        assert_bf16_close(Sf_gpu[bi:bi + 1], S_ref, f"layer core fused final state, row {bi}")
