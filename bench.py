@@ -537,6 +537,8 @@ def run_profile(mode, reps):
     decode     consecutive gdn_gates + gdn_recurrent_step calls on 256 sequences x 32 heads
     conv       gdn_causal_conv1d_silu on the [2, 16384, 8192] mix, then gdn_gated_rmsnorm on the
                v channels viewed as 128-wide rows
+    layercore  the layer core on B = 2 x 16384 tokens: gdn_causal_conv1d_silu, then
+               gdn_chunk_fwd_gated_norm on q, k, v read in place from the conv output
     """
     from gated_deltanet_fwd_b200 import gdn
     dev = torch.device("cuda", 0)
@@ -567,6 +569,19 @@ def run_profile(mode, reps):
         for _ in range(reps):
             y = gdn.gdn_causal_conv1d_silu(mix, cw, None, n_l2norm_ch=nqk, l2norm_group=w["dk"])
             gdn.gdn_gated_rmsnorm(y[:, :, nqk:].contiguous().view(-1, w["dv"]), z, nw)
+    elif mode == "layercore":
+        w = inputs.WORKLOADS["layer_core_2x16k"]
+        x = inputs.layer_core_inputs(**w, seed=1000 + w["index"])
+        B, T, Hk, Hv, d = w["B"], w["T"], w["Hk"], w["Hv"], w["dk"]
+        mix, cw = x["mix"].to(dev), x["conv_w"].to(dev)
+        a, b, z = x["a"].to(dev), x["b"].to(dev), x["z"].to(dev)
+        A_log, dt_bias, nw = x["A_log"].to(dev), x["dt_bias"].to(dev), x["norm_w"].to(dev)
+        for _ in range(reps):
+            y = gdn.gdn_causal_conv1d_silu(mix, cw, None, n_l2norm_ch=2 * Hk * d, l2norm_group=d)
+            gdn.gdn_chunk_fwd_gated_norm(y[:, :, :Hk * d].view(B, T, Hk, d),
+                                         y[:, :, Hk * d:2 * Hk * d].view(B, T, Hk, d),
+                                         y[:, :, 2 * Hk * d:].view(B, T, Hv, d), a, b, A_log,
+                                         dt_bias, z, nw, norm_eps=w["eps"])
     else:
         raise SystemExit(run_profile.__doc__)
     torch.cuda.synchronize()
@@ -584,7 +599,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--profile", default=None,
-                    help="run one workload for a profiler capture: prefill|prefill4k|decode|conv")
+                    help="run one workload for a profiler capture: "
+                         "prefill|prefill4k|decode|conv|layercore")
     ap.add_argument("--repeats", type=int, default=2, help="launches per --profile run")
     args = ap.parse_args()
     if args.profile:

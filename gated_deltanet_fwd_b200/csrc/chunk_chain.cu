@@ -37,6 +37,9 @@ namespace {
 
 using namespace ptx;
 
+// Warps: 0-3 the critical epilogues, 4-7 the side group, 8 the TMA producer, 9 the MMA issuer.
+// Ten warps over four SM sub-partitions put three on two of them, so a thread may hold at most
+// 168 registers.
 constexpr int CH_THREADS = 320;
 constexpr int W_PROD = 8, W_MMA = 9;
 
@@ -48,11 +51,10 @@ constexpr uint32_t ST_TP = 49152;      // [T'; P]: 128 rows x 128 B
 constexpr uint32_t ST_GD = 65536;      // Gamma[64], d[64] fp32
 constexpr uint32_t STAGE = 66560;      // 65 KB, a multiple of 1024
 constexpr uint32_t SM_GAM = 2 * STAGE;      // Gamma of the two chunks whose outputs are pending
-constexpr uint32_t SM_ROWS = SM_GAM + 512;   // fused norm: the chunk's outputs, 64 rows x 128 fp32
-constexpr uint32_t SM_Z = SM_ROWS + 32768;   // fused norm: the chunk's z gate, 128 x 128 B
-constexpr uint32_t SM_BAR = SM_Z + 16384;
-constexpr uint32_t SM_USED = SM_BAR + 256;
-constexpr uint32_t CH_SMEM = SM_USED + 1024;
+constexpr uint32_t SM_BAR = SM_GAM + 512;    // mbarriers, abort flag, tensor-memory slot
+// the request stays well below the SM's 228 KB, leaving the rest of the unified L1 / shared
+// memory to the L1 cache (which holds the side group's per-thread output staging)
+constexpr uint32_t CH_SMEM = SM_BAR + 256 + 1024;  // + slack for the 1024-byte alignment
 constexpr uint32_t STAGE_TX = 4 * 16384 + 512;
 static_assert(CH_SMEM <= 232448, "shared memory budget");
 static_assert(ST_V == ST_KQ + 32768 && ST_TP == ST_V + 16384, "stage layout");
@@ -60,7 +62,7 @@ static_assert(ST_V == ST_KQ + 32768 && ST_TP == ST_V + 16384, "stage layout");
 enum { B_FULL0 = 0, B_EMPTY0 = 2, B_K = 4, B_U = 5, B_S = 6, B_O = 7, B_DRAIN = 8, B_N = 9 };
 
 // named barriers: producer/consumer hand-offs to the MMA issuer and between the two groups
-enum { NB_X = 1, NB_U = 2, NB_S = 3, NB_SR = 4, NB_H = 5 };
+enum { NB_X = 1, NB_U = 2, NB_S = 3, NB_SR = 4 };
 constexpr int NB_ALL = 288;  // epilogue group + side group + issuer warp
 constexpr int NB_EI = 160;   // epilogue group + issuer warp
 constexpr int NB_EH = 256;   // epilogue group + side group
@@ -69,12 +71,12 @@ constexpr int NB_EH = 256;   // epilogue group + side group
 constexpr uint32_t TM_S = 0, TM_K = 128, TM_Q = 192, TM_U = 256, TM_SB = 320, TM_X = 384,
                    TM_UT = 416, TM_UD = 448;
 
-// Optional phase timing, compiled in only with -DGDN_CHAIN_TRACE: clock64 stamps of CTA 0, 16 slots
+// Optional phase timing, compiled in only with -DGDN_CHAIN_TRACE: clock64 stamps of CTA 0, 32 slots
 // per chunk, written to ChainParams::trace.
 #ifdef GDN_CHAIN_TRACE
 #define CH_TS(c, k)                                                            \
   do {                                                                         \
-    if (P.trace && blockIdx.x == 0 && (c) < 256) P.trace[(c) * 16 + (k)] = clock64(); \
+    if (P.trace && blockIdx.x == 0 && (c) < 256) P.trace[(c) * 32 + (k)] = clock64(); \
   } while (0)
 #else
 #define CH_TS(c, k) \
@@ -100,11 +102,6 @@ struct ChainParams {
   float* st;        // state arrays SOUT, BSEG, MSEG, SIN (scan phases only)
   int debug_skip_chunk;  // failure-test builds only: the producer withholds this chunk's tiles
   unsigned long long* trace;  // phase timing (trace builds only), else unused
-  // fused gated RMSNorm of the outputs (z set): out receives y = o rsqrt(mean o^2 + eps)
-  // (1 + w) silu(z) per (token, head)
-  const __nv_bfloat16* z;
-  const float* norm_w;
-  float norm_eps;
 };
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
@@ -125,8 +122,6 @@ __device__ __forceinline__ void ld64(uint32_t taddr, float (&v)[64]) {
   tmem_ld16(taddr + 48, *reinterpret_cast<float(*)[16]>(v + 48));
 }
 
-// 320 threads: ten warps over four SM sub-partitions put three warps on two of them, so a thread
-// may hold at most 168 registers.
 __global__ void __launch_bounds__(CH_THREADS, 1) chunk_chain_kernel(
     const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
     const __grid_constant__ CUtensorMap map_v, const __grid_constant__ CUtensorMap map_tp,
@@ -219,414 +214,326 @@ __global__ void __launch_bounds__(CH_THREADS, 1) chunk_chain_kernel(
   };
   auto chunk_t0 = [&](int c) { return s_beg + (int64_t)tm::C * c; };
 
-  if (warp == W_PROD) {
-    // ------------------------------------------------------------ TMA producer -------------
-    if (lane == 0) {
-      prefetch_tensormap(&map_q);
-      prefetch_tensormap(&map_k);
-      prefetch_tensormap(&map_v);
-      prefetch_tensormap(&map_tp);
-      int issued = 0;
-      for (int c = 0; c < nchunks; ++c) {
-        const int st = c & 1;
-        if (c >= 2 && !wait(B_EMPTY0 + st, ((c >> 1) & 1) ^ 1)) break;
-        if (*abort_flag) break;
-        const int32_t t0 = (int32_t)chunk_t0(c);
-        unsigned char* sp = smem + st * STAGE;
-        uint64_t* fb = &bars[B_FULL0 + st];
-        mbar_arrive_expect_tx(fb, zero_v ? STAGE_TX - 16384 : STAGE_TX);
-#ifdef GDN_FAULT_INJECTION
-        if (c == P.debug_skip_chunk) continue;  // nothing lands: the waits on this stage run out
-#endif
-        tma_load_3d(sp + ST_KQ, &map_k, fb, 0, hk, t0);
-        tma_load_3d(sp + ST_KQ + 8192, &map_q, fb, 0, hk, t0);
-        tma_load_3d(sp + ST_KQ + 16384, &map_k, fb, 64, hk, t0);
-        tma_load_3d(sp + ST_KQ + 24576, &map_q, fb, 64, hk, t0);
-        if (!zero_v) {
-          tma_load_3d(sp + ST_V, &map_v, fb, 0, h, t0);
-          tma_load_3d(sp + ST_V + 8192, &map_v, fb, 64, h, t0);
-        }
-        const int64_t slot = slot0 + c;
-        tma_load_2d(sp + ST_TP, &map_tp, fb, 0, (int32_t)((slot * P.Hv + h) * 128));
-        bulk_load(sp + ST_GD, P.ws + P.gd_off + ((size_t)slot * P.Hv + h) * tm::GD_BYTES,
-                  tm::GD_BYTES, fb);
-        issued = c + 1;
-      }
-      // never leave the CTA with copies still landing in shared memory (each wait bounded; a
-      // stage whose copies were never issued simply runs out)
-      for (int c = issued - 2 < 0 ? 0 : issued - 2; c < issued; ++c)
-        if (!mbar_wait(&bars[B_FULL0 + (c & 1)], (uint32_t)(c >> 1) & 1))
-          report(P.status, GDN_ERR_TIMEOUT);
-    }
-  } else if (warp == W_MMA) {
-    // ------------------------------------------------------------ MMA issuer ---------------
-    const uint32_t id_n64 = idesc_bf16(128, 64, 0, 0);   // A tensor memory, B K-major
-    const uint32_t id_kq = idesc_bf16(128, 128, 0, 0);   // A tensor memory, B = [K; Q] K-major
-    const uint32_t id_v = idesc_bf16(128, 64, 1, 0);     // A = V^T (MN-major smem), B K-major
-    const uint32_t id_s = idesc_bf16(128, 128, 0, 1);    // B = K (MN-major)
-    named_bar(NB_S, NB_ALL);  // S and its bf16 copy initialised; D_q free
-    for (int c = 0; c < nchunks; ++c) {
-      const int st = c & 1;
-      const uint32_t sp = sbase + st * STAGE;
-      if (lane == 0) CH_TS(c, 0);
-      const bool have = wait(B_FULL0 + st, (c >> 1) & 1);
-      if (c > 0) named_bar(NB_S, NB_ALL);  // refresh of S done, D_q read
-      if (lane == 0) CH_TS(c, 1);
-      const bool go = have && !*abort_flag;
-      const bool leader = lane == 0;
-      const uint64_t dKQ = sdesc_sw128(sp + ST_KQ, 16, 1024);    // [K; Q] as K-major B
-      const uint64_t dVt = sdesc_sw128(sp + ST_V, 8192, 1024);   // V^T as MN-major A
-      const uint64_t dTp = sdesc_sw128(sp + ST_TP, 16, 1024);    // T' as K-major B
-      const uint64_t dP = sdesc_sw128(sp + ST_TP + 8192, 16, 1024);  // P as K-major B
-      const uint64_t dKn = sdesc_sw128(sp + ST_KQ, 16384, 1024);  // K as MN-major B
-      if (go && leader) {
-        tc_fence_after();
+  if (warp < 8) {
+    if (warp < 4) {
+      // ------------------------------------------------------------ critical epilogues -------
+      const int j = 32 * warp + lane;  // value row of S = tensor-memory lane
+      const uint32_t lo = (uint32_t)(32 * warp) << 16;
+      // initial state: fp32 master and bf16 operand copy
+      {
+        const float* src = src_state ? src_state + (size_t)j * tm::D : nullptr;
 #pragma unroll
-        for (int ks = 0; ks < 8; ++ks)
-          mma_bf16_ts(tmem + TM_K, tmem + TM_SB + 8 * ks,
-                      dadd(dKQ, (ks >> 2) * 16384 + (ks & 3) * 32), id_kq, ks > 0);
-        mma_commit(&bars[B_K]);
-        if (!zero_v) {
+        for (int blk = 0; blk < 4; ++blk) {  // 32 columns at a time
+          float v[32];
 #pragma unroll
-          for (int ks = 0; ks < 4; ++ks)
-            mma_bf16_ss(tmem + TM_U, dadd(dVt, ks * 2048), dadd(dTp, ks * 32), id_v, ks > 0);
-        }
-      }
-      if (lane == 0) CH_TS(c, 2);
-      __syncwarp();
-      named_bar(NB_X, NB_EI);  // X' written
-      if (lane == 0) CH_TS(c, 3);
-      if (go && leader && !*abort_flag) {
-        tc_fence_after();
+          for (int q4 = 0; q4 < 8; ++q4) {
+            const float4 f = src ? __ldg(reinterpret_cast<const float4*>(src + 32 * blk) + q4)
+                                 : make_float4(0.f, 0.f, 0.f, 0.f);
+            v[4 * q4] = f.x;
+            v[4 * q4 + 1] = f.y;
+            v[4 * q4 + 2] = f.z;
+            v[4 * q4 + 3] = f.w;
+          }
+          if (ident) {
 #pragma unroll
-        for (int ks = 0; ks < 4; ++ks)
-          mma_bf16_ts(tmem + TM_U, tmem + TM_X + 8 * ks, dadd(dTp, ks * 32), id_n64,
-                      !zero_v || ks > 0);
-        mma_commit(&bars[B_U]);
-      }
-      __syncwarp();
-      named_bar(NB_U, NB_ALL);  // U^T, U^T diag(d) written; S scaled by Gamma_63
-      if (lane == 0) CH_TS(c, 4);
-      if (go && leader && !*abort_flag) {
-        tc_fence_after();
-#pragma unroll
-        for (int ks = 0; ks < 4; ++ks)
-          mma_bf16_ts(tmem + TM_S, tmem + TM_UD + 8 * ks, dadd(dKn, ks * 2048), id_s, 1);
-        mma_commit(&bars[B_S]);
-        if (has_out) {
-#pragma unroll
-          for (int ks = 0; ks < 4; ++ks)
-            mma_bf16_ts(tmem + TM_K, tmem + TM_UT + 8 * ks, dadd(dP, ks * 32), id_n64, ks > 0);
-          mma_commit(&bars[B_O]);
-        }
-        mma_commit(&bars[B_EMPTY0 + st]);
-      }
-      __syncwarp();
-    }
-    if (lane == 0) {
-      // every MMA has completed before tensor memory is read back or released
-      mma_commit(&bars[B_DRAIN]);
-      if (!mbar_wait(&bars[B_DRAIN], 0)) fail(GDN_ERR_TIMEOUT);
-    }
-  } else if (warp < 4) {
-    // ------------------------------------------------------------ critical epilogues -------
-    const int j = 32 * warp + lane;  // value row of S = tensor-memory lane
-    const uint32_t lo = (uint32_t)(32 * warp) << 16;
-    // initial state: fp32 master and bf16 operand copy
-    {
-      const float* src = src_state ? src_state + (size_t)j * tm::D : nullptr;
-#pragma unroll
-      for (int blk = 0; blk < 4; ++blk) {  // 32 columns at a time
-        float v[32];
-#pragma unroll
-        for (int q4 = 0; q4 < 8; ++q4) {
-          const float4 f = src ? __ldg(reinterpret_cast<const float4*>(src + 32 * blk) + q4)
-                               : make_float4(0.f, 0.f, 0.f, 0.f);
-          v[4 * q4] = f.x;
-          v[4 * q4 + 1] = f.y;
-          v[4 * q4 + 2] = f.z;
-          v[4 * q4 + 3] = f.w;
-        }
-        if (ident) {
-#pragma unroll
-          for (int q = 0; q < 32; ++q) v[q] = (32 * blk + q == j) ? 1.0f : 0.0f;
-        }
-        tmem_st16(tmem + lo + TM_S + 32 * blk, *reinterpret_cast<float(*)[16]>(v));
-        tmem_st16(tmem + lo + TM_S + 32 * blk + 16, *reinterpret_cast<float(*)[16]>(v + 16));
-        uint32_t pk[16];
-#pragma unroll
-        for (int q = 0; q < 16; ++q) pk[q] = pack_bf16x2(v[2 * q], v[2 * q + 1]);
-        tmem_st16u(tmem + lo + TM_SB + 16 * blk, pk);
-      }
-      tmem_st_wait();
-      tc_fence_before();
-      named_bar_arrive(NB_SR, NB_EH);  // the side group may now scale S
-      named_bar(NB_S, NB_ALL);
-    }
-    for (int c = 0; c < nchunks; ++c) {
-      const int st = c & 1;
-      const float* gd = reinterpret_cast<const float*>(smem + st * STAGE + ST_GD);
-      wait(B_FULL0 + st, (c >> 1) & 1);  // the chunk's Gamma and d are visible to this thread
-      // ---- X' = -(S K^T) diag(Gamma), 32 columns at a time
-      if (wait(B_K, c & 1)) {
-        if (tid == 0) CH_TS(c, 5);
-        tc_fence_after();
-        float dk[64];
-        ld64(tmem + lo + TM_K, dk);
-        tmem_ld_wait();
-#pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
+            for (int q = 0; q < 32; ++q) v[q] = (32 * blk + q == j) ? 1.0f : 0.0f;
+          }
+          tmem_st16(tmem + lo + TM_S + 32 * blk, *reinterpret_cast<float(*)[16]>(v));
+          tmem_st16(tmem + lo + TM_S + 32 * blk + 16, *reinterpret_cast<float(*)[16]>(v + 16));
           uint32_t pk[16];
 #pragma unroll
-          for (int q4 = 0; q4 < 8; ++q4) {
-            const float4 gm = *reinterpret_cast<const float4*>(gd + 32 * hh + 4 * q4);
-            const float* x = dk + 32 * hh + 4 * q4;
-            pk[2 * q4] = pack_bf16x2(-gm.x * x[0], -gm.y * x[1]);
-            pk[2 * q4 + 1] = pack_bf16x2(-gm.z * x[2], -gm.w * x[3]);
-          }
-          tmem_st16u(tmem + lo + TM_X + 16 * hh, pk);
+          for (int q = 0; q < 16; ++q) pk[q] = pack_bf16x2(v[2 * q], v[2 * q + 1]);
+          tmem_st16u(tmem + lo + TM_SB + 16 * blk, pk);
         }
         tmem_st_wait();
+        tc_fence_before();
+        named_bar_arrive(NB_SR, NB_EH);  // the side group may now scale S
+        named_bar(NB_S, NB_ALL);
       }
-      if (tid == 0) CH_TS(c, 6);
-      tc_fence_before();
-      named_bar_arrive(NB_X, NB_EI);
-      // ---- U^T and U^T diag(d)
-      if (wait(B_U, c & 1)) {
-        if (tid == 0) CH_TS(c, 7);
-        tc_fence_after();
-        float u[64];
-        ld64(tmem + lo + TM_U, u);
-        tmem_ld_wait();
+      for (int c = 0; c < nchunks; ++c) {
+        const int st = c & 1;
+        const float* gd = reinterpret_cast<const float*>(smem + st * STAGE + ST_GD);
+        wait(B_FULL0 + st, (c >> 1) & 1);  // the chunk's Gamma and d are visible to this thread
+        // ---- X' = -(S K^T) diag(Gamma), 32 columns at a time
+        if (wait(B_K, c & 1)) {
+          if (tid == 0) CH_TS(c, 5);
+          tc_fence_after();
+          float dk[64];
+          ld64(tmem + lo + TM_K, dk);
+          tmem_ld_wait();
 #pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-          uint32_t pk[16], pd[16];
+          for (int hh = 0; hh < 2; ++hh) {
+            uint32_t pk[16];
 #pragma unroll
-          for (int q4 = 0; q4 < 8; ++q4) {
-            const float4 dd = *reinterpret_cast<const float4*>(gd + 64 + 32 * hh + 4 * q4);
-            const float* x = u + 32 * hh + 4 * q4;
-            pk[2 * q4] = pack_bf16x2(x[0], x[1]);
-            pk[2 * q4 + 1] = pack_bf16x2(x[2], x[3]);
-            pd[2 * q4] = pack_bf16x2(x[0] * dd.x, x[1] * dd.y);
-            pd[2 * q4 + 1] = pack_bf16x2(x[2] * dd.z, x[3] * dd.w);
+            for (int q4 = 0; q4 < 8; ++q4) {
+              const float4 gm = *reinterpret_cast<const float4*>(gd + 32 * hh + 4 * q4);
+              const float* x = dk + 32 * hh + 4 * q4;
+              pk[2 * q4] = pack_bf16x2(-gm.x * x[0], -gm.y * x[1]);
+              pk[2 * q4 + 1] = pack_bf16x2(-gm.z * x[2], -gm.w * x[3]);
+            }
+            tmem_st16u(tmem + lo + TM_X + 16 * hh, pk);
           }
-          tmem_st16u(tmem + lo + TM_UT + 16 * hh, pk);
-          tmem_st16u(tmem + lo + TM_UD + 16 * hh, pd);
+          tmem_st_wait();
         }
-        tmem_st_wait();
-      }
-      tc_fence_before();
-      // a full barrier, not an arrival: the group then never runs a barrier instance ahead of
-      // the issuer, even when an abort makes it skip its waits
-      if (tid == 0) CH_TS(c, 8);
-      named_bar(NB_U, NB_ALL);
-      if (tid == 0) CH_TS(c, 9);
-      // ---- refresh of the bf16 copy of the new state (not after the last chunk)
-      const bool s_ok = wait(B_S, c & 1);
-      if (tid == 0) CH_TS(c, 10);
-      if (c + 1 < nchunks) {
-        if (s_ok) {
+        if (tid == 0) CH_TS(c, 6);
+        tc_fence_before();
+        named_bar_arrive(NB_X, NB_EI);
+        // ---- U^T and U^T diag(d)
+        if (wait(B_U, c & 1)) {
+          if (tid == 0) CH_TS(c, 7);
           tc_fence_after();
 #pragma unroll
           for (int hh = 0; hh < 2; ++hh) {
-            float v[64];
-            ld64(tmem + lo + TM_S + 64 * hh, v);
+            float u[32];
+            tmem_ld32(tmem + lo + TM_U + 32 * hh, u);
             tmem_ld_wait();
-            uint32_t pk[32];
+            uint32_t pk[16], pd[16];
 #pragma unroll
-            for (int q = 0; q < 32; ++q) pk[q] = pack_bf16x2(v[2 * q], v[2 * q + 1]);
-            tmem_st16u(tmem + lo + TM_SB + 32 * hh, *reinterpret_cast<uint32_t(*)[16]>(pk));
-            tmem_st16u(tmem + lo + TM_SB + 32 * hh + 16,
-                       *reinterpret_cast<uint32_t(*)[16]>(pk + 16));
+            for (int q4 = 0; q4 < 8; ++q4) {
+              const float4 dd = *reinterpret_cast<const float4*>(gd + 64 + 32 * hh + 4 * q4);
+              const float* x = u + 4 * q4;
+              pk[2 * q4] = pack_bf16x2(x[0], x[1]);
+              pk[2 * q4 + 1] = pack_bf16x2(x[2], x[3]);
+              pd[2 * q4] = pack_bf16x2(x[0] * dd.x, x[1] * dd.y);
+              pd[2 * q4 + 1] = pack_bf16x2(x[2] * dd.z, x[3] * dd.w);
+            }
+            tmem_st16u(tmem + lo + TM_UT + 16 * hh, pk);
+            tmem_st16u(tmem + lo + TM_UD + 16 * hh, pd);
           }
+          tmem_st_wait();
         }
         tc_fence_before();
-        named_bar_arrive(NB_SR, NB_EH);  // S read: the side group may scale it
+        // a full barrier, not an arrival: the group then never runs a barrier instance ahead of
+        // the issuer, even when an abort makes it skip its waits
+        if (tid == 0) CH_TS(c, 8);
+        named_bar(NB_U, NB_ALL);
+        if (tid == 0) CH_TS(c, 9);
+        // ---- refresh of the bf16 copy of the new state (not after the last chunk)
+        const bool s_ok = wait(B_S, c & 1);
+        if (tid == 0) CH_TS(c, 10);
+        if (c + 1 < nchunks) {
+          if (s_ok) {
+            tc_fence_after();
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+              float v[64];
+              ld64(tmem + lo + TM_S + 64 * hh, v);
+              tmem_ld_wait();
+              uint32_t pk[32];
+#pragma unroll
+              for (int q = 0; q < 32; ++q) pk[q] = pack_bf16x2(v[2 * q], v[2 * q + 1]);
+              tmem_st16u(tmem + lo + TM_SB + 32 * hh, *reinterpret_cast<uint32_t(*)[16]>(pk));
+              tmem_st16u(tmem + lo + TM_SB + 32 * hh + 16,
+                         *reinterpret_cast<uint32_t(*)[16]>(pk + 16));
+            }
+          }
+          tc_fence_before();
+          named_bar_arrive(NB_SR, NB_EH);  // S read: the side group may scale it
+          tmem_st_wait();
+          if (tid == 0) CH_TS(c, 11);
+          tc_fence_before();
+          named_bar(NB_S, NB_ALL);
+        }
+
+      }
+    } else {
+      // ------------------------------------------------------------ side group (warps 4-7) ---
+      const int t4 = tid - 128;
+      const int j = 32 * (warp - 4) + lane;
+      const uint32_t lo = (uint32_t)(32 * (warp - 4)) << 16;
+      // Gamma of the chunks whose outputs are pending (the stage may be refilled before then)
+      float* gam_o = reinterpret_cast<float*>(smem + SM_GAM);
+      // S <- Gamma_63(c) S in tensor memory (after the critical group has read S); keeps Gamma(c)
+      auto scale_s = [&](int c) {
+        named_bar(NB_SR, NB_EH);
+        tc_fence_after();
+        if (!wait(B_FULL0 + (c & 1), (c >> 1) & 1)) return;
+        const float* gd = reinterpret_cast<const float*>(smem + (c & 1) * STAGE + ST_GD);
+        if (t4 < 64) gam_o[(c & 1) * 64 + t4] = gd[t4];
+        const float gl = gd[63];
+#pragma unroll
+        for (int hh = 0; hh < 4; ++hh) {
+          float v[32];
+          tmem_ld32(tmem + lo + TM_S + 32 * hh, v);
+          tmem_ld_wait();
+#pragma unroll
+          for (int q = 0; q < 32; ++q) v[q] *= gl;
+#pragma unroll
+          for (int q4 = 0; q4 < 2; ++q4)
+            tmem_st16(tmem + lo + TM_S + 32 * hh + 16 * q4, *reinterpret_cast<float(*)[16]>(v + 16 * q4));
+        }
         tmem_st_wait();
-        if (tid == 0) CH_TS(c, 11);
-        tc_fence_before();
-        named_bar(NB_S, NB_ALL);
-      }
-    }
-  } else {
-    // ------------------------------------------------------------ side group (warps 4-7) ---
-    const int t4 = tid - 128;
-    const int j = 32 * (warp - 4) + lane;
-    const uint32_t lo = (uint32_t)(32 * (warp - 4)) << 16;
-    // Gamma of the chunks whose outputs are pending (the stage may be refilled before then)
-    float* gam_o = reinterpret_cast<float*>(smem + SM_GAM);
-    // S <- Gamma_63(c) S in tensor memory (after the critical group has read S); keeps Gamma(c)
-    auto scale_s = [&](int c) {
-      named_bar(NB_SR, NB_EH);
-      tc_fence_after();
-      if (!wait(B_FULL0 + (c & 1), (c >> 1) & 1)) return;
-      const float* gd = reinterpret_cast<const float*>(smem + (c & 1) * STAGE + ST_GD);
-      if (t4 < 64) gam_o[(c & 1) * 64 + t4] = gd[t4];
-      const float gl = gd[63];
-#pragma unroll
-      for (int hh = 0; hh < 4; ++hh) {
-        float v[32];
-        tmem_ld32(tmem + lo + TM_S + 32 * hh, v);
-        tmem_ld_wait();
-#pragma unroll
-        for (int q = 0; q < 32; ++q) v[q] *= gl;
-#pragma unroll
-        for (int q4 = 0; q4 < 2; ++q4)
-          tmem_st16(tmem + lo + TM_S + 32 * hh + 16 * q4, *reinterpret_cast<float(*)[16]>(v + 16 * q4));
-      }
-      tmem_st_wait();
-    };
-    named_bar_arrive(NB_S, NB_ALL);  // D_q is free
-    scale_s(0);
-    tc_fence_before();
-    // fused norm: thread t4 owns half `half` of token row r of each chunk; its 128 bytes of z are
-    // copied into its own slot of SM_Z at the top of the chunk (the 16-byte pieces in an order
-    // rotated by t4, so that eight neighbouring threads hit eight different bank groups)
-    unsigned char* zs = smem + SM_Z + t4 * 128;
-    const int zr_row = t4 >> 1, zr_half = t4 & 1;
-    for (int c = 0; c < nchunks; ++c) {
-      if (P.z && has_out) {
-        const int64_t t0 = chunk_t0(c);
-        if (zr_row < (int)min((int64_t)tm::C, s_end - t0)) {
-          const __nv_bfloat16* zrow =
-              P.z + ((size_t)(t0 + zr_row) * P.Hv + h) * tm::D + 64 * zr_half;
-#pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            const int cc = (i + t4) & 7;
-            cp_async16(zs + 16 * cc, zrow + 8 * cc);
-          }
-        }
-      }
-      named_bar(NB_U, NB_ALL);  // S scaled by Gamma_63(c); a full barrier (see the other group)
-      if (P.z) {
-        // ---- outputs of chunk c with the gated RMSNorm: O^T = diag(Gamma) (S Q^T) + U^T P^T is
-        // staged as [row][column] fp32, then each thread takes half of a token row: its sum of
-        // squares (with the other half's), the z gate and the norm weight, and 64 bytes of y
-        float* rows = reinterpret_cast<float*>(smem + SM_ROWS);
-        named_bar(NB_H, 128);  // the previous chunk's rows have been read
+      };
+      named_bar_arrive(NB_S, NB_ALL);  // D_q is free
+      scale_s(0);
+      tc_fence_before();
+      for (int c = 0; c < nchunks; ++c) {
+        named_bar(NB_U, NB_ALL);  // S scaled by Gamma_63(c); a full barrier (see the other group)
+        // ---- outputs of chunk c: O^T = diag(Gamma) (S Q^T) + U^T P^T, held as scaled bf16 pairs
+        // (rows 2q, 2q + 1) of value column j
+        uint32_t ob[32];
         const bool o_ok = has_out && wait(B_O, c & 1);
         if (t4 == 0) CH_TS(c, 12);
         if (o_ok) {
           tc_fence_after();
           const float* gm = gam_o + (c & 1) * 64;
-          float* col = rows + j;
-#pragma unroll 1
-          for (int q16 = 0; q16 < 4; ++q16) {
-            float dq[16], doo[16];
-            tmem_ld16(tmem + lo + TM_Q + 16 * q16, dq);
-            tmem_ld16(tmem + lo + TM_K + 16 * q16, doo);
+#pragma unroll
+          for (int hh = 0; hh < 2; ++hh) {
+            float dq[32], doo[32];
+            tmem_ld16(tmem + lo + TM_Q + 32 * hh, *reinterpret_cast<float(*)[16]>(dq));
+            tmem_ld16(tmem + lo + TM_Q + 32 * hh + 16, *reinterpret_cast<float(*)[16]>(dq + 16));
+            tmem_ld16(tmem + lo + TM_K + 32 * hh, *reinterpret_cast<float(*)[16]>(doo));
+            tmem_ld16(tmem + lo + TM_K + 32 * hh + 16, *reinterpret_cast<float(*)[16]>(doo + 16));
             tmem_ld_wait();
 #pragma unroll
-            for (int q = 0; q < 16; ++q)
-              col[(16 * q16 + q) * 128] = P.scale * fmaf(gm[16 * q16 + q], dq[q], doo[q]);
+            for (int q = 0; q < 16; ++q) {
+              const float2 g2 = *reinterpret_cast<const float2*>(gm + 32 * hh + 2 * q);
+              ob[16 * hh + q] = pack_bf16x2(P.scale * fmaf(g2.x, dq[2 * q], doo[2 * q]),
+                                            P.scale * fmaf(g2.y, dq[2 * q + 1], doo[2 * q + 1]));
+            }
           }
         }
         tc_fence_before();
         if (c + 1 < nchunks) named_bar_arrive(NB_S, NB_ALL);  // D_q and D_o read
-        named_bar(NB_H, 128);  // the chunk's rows are complete
         // ---- S scaled by Gamma_63 for chunk c + 1 (needed before the issuer's next NB_U)
         if (c + 1 < nchunks) {
           scale_s(c + 1);
           if (t4 == 0) CH_TS(c, 14);
           tc_fence_before();
         }
-        cp_async_wait_all();  // this thread's z pieces of chunk c
         if (o_ok && !*abort_flag) {
+          // lanes j, j ^ 1 swap halves: an even lane stores row 2q at columns j, j + 1, an odd lane
+          // row 2q + 1 at columns j - 1, j -- each store a 4-byte pair, each warp store two
+          // contiguous 64-byte row segments
           const int64_t t0 = chunk_t0(c);
           const int L = (int)min((int64_t)tm::C, s_end - t0);
-          const int r = zr_row, half = zr_half;
-          // float4 q of the half row, read in an order rotated by t4 (bank groups as for z)
-          const float4* xr = reinterpret_cast<const float4*>(rows + r * 128 + 64 * half);
-          float ssq = 0.0f;
-#pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const float4 x = xr[(i + t4) & 15];
-            ssq = fmaf(x.x, x.x, fmaf(x.y, x.y, fmaf(x.z, x.z, fmaf(x.w, x.w, ssq))));
-          }
-          ssq += __shfl_xor_sync(0xffffffffu, ssq, 1);
-          const float inv = rsqrtf(ssq * (1.0f / tm::D) + P.norm_eps);
-          if (r < L) {
-            const size_t off = ((size_t)(t0 + r) * P.Hv + h) * tm::D + 64 * half;
-            uint4* yr = reinterpret_cast<uint4*>(P.out + off);
-            const float* wh = P.norm_w + 64 * half;
-#pragma unroll 1
-            for (int i = 0; i < 8; ++i) {
-              const int cc = (i + t4) & 7;
-              const uint4 zu = *reinterpret_cast<const uint4*>(zs + 16 * cc);
-              const uint32_t zw[4] = {zu.x, zu.y, zu.z, zu.w};
-              const float4 x0 = xr[2 * cc], x1 = xr[2 * cc + 1];
-              const float xv[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
-              const float4 w0 = __ldg(reinterpret_cast<const float4*>(wh + 8 * cc));
-              const float4 w1 = __ldg(reinterpret_cast<const float4*>(wh + 8 * cc + 4));
-              const float wv[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
-              uint32_t pk[4];
-#pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                const float2 zz = make_float2(__uint_as_float(zw[e] << 16),
-                                              __uint_as_float(zw[e] & 0xffff0000u));
-                pk[e] = pack_bf16x2(xv[2 * e] * inv * (1.0f + wv[2 * e]) * siluf_(zz.x),
-                                    xv[2 * e + 1] * inv * (1.0f + wv[2 * e + 1]) * siluf_(zz.y));
-              }
-              yr[cc] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-            }
+          const int odd = j & 1;
+          const int64_t rs = (int64_t)P.Hv * tm::D;  // elements between consecutive tokens
+          uint32_t* dst = reinterpret_cast<uint32_t*>(P.out + (t0 + odd) * rs + h * tm::D + (j & ~1));
+          const uint32_t sel = odd ? 0x7632u : 0x5410u;
+          const int64_t step = rs;  // two token rows of bf16, counted in 4-byte units
+#pragma unroll 8
+          for (int q = 0; q < 32; ++q) {
+            const uint32_t mine = ob[q];
+            const uint32_t other = __shfl_xor_sync(0xffffffffu, mine, 1);
+            const uint32_t pair = odd ? __byte_perm(other, mine, sel) : __byte_perm(mine, other, sel);
+            if (2 * q + odd < L) *dst = pair;
+            dst += step;
           }
         }
         if (t4 == 0) CH_TS(c, 13);
-        continue;
       }
-      // ---- outputs of chunk c: O^T = diag(Gamma) (S Q^T) + U^T P^T, held as scaled bf16 pairs
-      // (rows 2q, 2q + 1) of value column j
-      uint32_t ob[32];
-      const bool o_ok = has_out && wait(B_O, c & 1);
-      if (t4 == 0) CH_TS(c, 12);
-      if (o_ok) {
-        tc_fence_after();
-        const float* gm = gam_o + (c & 1) * 64;
+    }
+  } else {
+    if (warp == W_PROD) {
+      // ------------------------------------------------------------ TMA producer -------------
+      if (lane == 0) {
+        prefetch_tensormap(&map_q);
+        prefetch_tensormap(&map_k);
+        prefetch_tensormap(&map_v);
+        prefetch_tensormap(&map_tp);
+        int issued = 0;
+        for (int c = 0; c < nchunks; ++c) {
+          const int st = c & 1;
+          if (c >= 2 && !wait(B_EMPTY0 + st, ((c >> 1) & 1) ^ 1)) break;
+          if (*abort_flag) break;
+          const int32_t t0 = (int32_t)chunk_t0(c);
+          unsigned char* sp = smem + st * STAGE;
+          uint64_t* fb = &bars[B_FULL0 + st];
+          mbar_arrive_expect_tx(fb, zero_v ? STAGE_TX - 16384 : STAGE_TX);
+  #ifdef GDN_FAULT_INJECTION
+          if (c == P.debug_skip_chunk) continue;  // nothing lands: the waits on this stage run out
+  #endif
+          tma_load_3d(sp + ST_KQ, &map_k, fb, 0, hk, t0);
+          tma_load_3d(sp + ST_KQ + 8192, &map_q, fb, 0, hk, t0);
+          tma_load_3d(sp + ST_KQ + 16384, &map_k, fb, 64, hk, t0);
+          tma_load_3d(sp + ST_KQ + 24576, &map_q, fb, 64, hk, t0);
+          if (!zero_v) {
+            tma_load_3d(sp + ST_V, &map_v, fb, 0, h, t0);
+            tma_load_3d(sp + ST_V + 8192, &map_v, fb, 64, h, t0);
+          }
+          const int64_t slot = slot0 + c;
+          tma_load_2d(sp + ST_TP, &map_tp, fb, 0, (int32_t)((slot * P.Hv + h) * 128));
+          bulk_load(sp + ST_GD, P.ws + P.gd_off + ((size_t)slot * P.Hv + h) * tm::GD_BYTES,
+                    tm::GD_BYTES, fb);
+          issued = c + 1;
+        }
+        // never leave the CTA with copies still landing in shared memory (each wait bounded; a
+        // stage whose copies were never issued simply runs out)
+        for (int c = issued - 2 < 0 ? 0 : issued - 2; c < issued; ++c)
+          if (!mbar_wait(&bars[B_FULL0 + (c & 1)], (uint32_t)(c >> 1) & 1))
+            report(P.status, GDN_ERR_TIMEOUT);
+      }
+    } else if (warp == W_MMA) {
+      // ------------------------------------------------------------ MMA issuer ---------------
+      const uint32_t id_n64 = idesc_bf16(128, 64, 0, 0);   // A tensor memory, B K-major
+      const uint32_t id_kq = idesc_bf16(128, 128, 0, 0);   // A tensor memory, B = [K; Q] K-major
+      const uint32_t id_v = idesc_bf16(128, 64, 1, 0);     // A = V^T (MN-major smem), B K-major
+      const uint32_t id_s = idesc_bf16(128, 128, 0, 1);    // B = K (MN-major)
+      named_bar(NB_S, NB_ALL);  // S and its bf16 copy initialised; D_q free
+      for (int c = 0; c < nchunks; ++c) {
+        const int st = c & 1;
+        const uint32_t sp = sbase + st * STAGE;
+        if (lane == 0) CH_TS(c, 0);
+        const bool have = wait(B_FULL0 + st, (c >> 1) & 1);
+        if (c > 0) named_bar(NB_S, NB_ALL);  // refresh of S done, D_q read
+        if (lane == 0) CH_TS(c, 1);
+        const bool go = have && !*abort_flag;
+        const bool leader = lane == 0;
+        const uint64_t dKQ = sdesc_sw128(sp + ST_KQ, 16, 1024);    // [K; Q] as K-major B
+        const uint64_t dVt = sdesc_sw128(sp + ST_V, 8192, 1024);   // V^T as MN-major A
+        const uint64_t dTp = sdesc_sw128(sp + ST_TP, 16, 1024);    // T' as K-major B
+        const uint64_t dP = sdesc_sw128(sp + ST_TP + 8192, 16, 1024);  // P as K-major B
+        const uint64_t dKn = sdesc_sw128(sp + ST_KQ, 16384, 1024);  // K as MN-major B
+        if (go && leader) {
+          tc_fence_after();
 #pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-          float dq[32], doo[32];
-          tmem_ld16(tmem + lo + TM_Q + 32 * hh, *reinterpret_cast<float(*)[16]>(dq));
-          tmem_ld16(tmem + lo + TM_Q + 32 * hh + 16, *reinterpret_cast<float(*)[16]>(dq + 16));
-          tmem_ld16(tmem + lo + TM_K + 32 * hh, *reinterpret_cast<float(*)[16]>(doo));
-          tmem_ld16(tmem + lo + TM_K + 32 * hh + 16, *reinterpret_cast<float(*)[16]>(doo + 16));
-          tmem_ld_wait();
+          for (int ks = 0; ks < 8; ++ks)
+            mma_bf16_ts(tmem + TM_K, tmem + TM_SB + 8 * ks,
+                        dadd(dKQ, (ks >> 2) * 16384 + (ks & 3) * 32), id_kq, ks > 0);
+          mma_commit(&bars[B_K]);
+          if (!zero_v) {
 #pragma unroll
-          for (int q = 0; q < 16; ++q) {
-            const float2 g2 = *reinterpret_cast<const float2*>(gm + 32 * hh + 2 * q);
-            ob[16 * hh + q] = pack_bf16x2(P.scale * fmaf(g2.x, dq[2 * q], doo[2 * q]),
-                                          P.scale * fmaf(g2.y, dq[2 * q + 1], doo[2 * q + 1]));
+            for (int ks = 0; ks < 4; ++ks)
+              mma_bf16_ss(tmem + TM_U, dadd(dVt, ks * 2048), dadd(dTp, ks * 32), id_v, ks > 0);
           }
         }
-      }
-      tc_fence_before();
-      if (c + 1 < nchunks) named_bar_arrive(NB_S, NB_ALL);  // D_q and D_o read
-      // ---- S scaled by Gamma_63 for chunk c + 1 (needed before the issuer's next NB_U)
-      if (c + 1 < nchunks) {
-        scale_s(c + 1);
-        if (t4 == 0) CH_TS(c, 14);
-        tc_fence_before();
-      }
-      if (o_ok && !*abort_flag) {
-        // lanes j, j ^ 1 swap halves: an even lane stores row 2q at columns j, j + 1, an odd lane
-        // row 2q + 1 at columns j - 1, j -- each store a 4-byte pair, each warp store two
-        // contiguous 64-byte row segments
-        const int64_t t0 = chunk_t0(c);
-        const int L = (int)min((int64_t)tm::C, s_end - t0);
-        const int odd = j & 1;
-        const int64_t rs = (int64_t)P.Hv * tm::D;  // elements between consecutive tokens
-        uint32_t* dst = reinterpret_cast<uint32_t*>(P.out + (t0 + odd) * rs + h * tm::D + (j & ~1));
-        const uint32_t sel = odd ? 0x7632u : 0x5410u;
-        const int64_t step = rs;  // two token rows of bf16, counted in 4-byte units
-#pragma unroll 8
-        for (int q = 0; q < 32; ++q) {
-          const uint32_t mine = ob[q];
-          const uint32_t other = __shfl_xor_sync(0xffffffffu, mine, 1);
-          const uint32_t pair = odd ? __byte_perm(other, mine, sel) : __byte_perm(mine, other, sel);
-          if (2 * q + odd < L) *dst = pair;
-          dst += step;
+        if (lane == 0) CH_TS(c, 2);
+        __syncwarp();
+        named_bar(NB_X, NB_EI);  // X' written
+        if (lane == 0) CH_TS(c, 3);
+        if (go && leader && !*abort_flag) {
+          tc_fence_after();
+#pragma unroll
+          for (int ks = 0; ks < 4; ++ks)
+            mma_bf16_ts(tmem + TM_U, tmem + TM_X + 8 * ks, dadd(dTp, ks * 32), id_n64,
+                        !zero_v || ks > 0);
+          mma_commit(&bars[B_U]);
         }
+        __syncwarp();
+        named_bar(NB_U, NB_ALL);  // U^T, U^T diag(d) written; S scaled by Gamma_63
+        if (lane == 0) CH_TS(c, 4);
+        if (go && leader && !*abort_flag) {
+          tc_fence_after();
+#pragma unroll
+          for (int ks = 0; ks < 4; ++ks)
+            mma_bf16_ts(tmem + TM_S, tmem + TM_UD + 8 * ks, dadd(dKn, ks * 2048), id_s, 1);
+          mma_commit(&bars[B_S]);
+          if (has_out) {
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks)
+              mma_bf16_ts(tmem + TM_K, tmem + TM_UT + 8 * ks, dadd(dP, ks * 32), id_n64, ks > 0);
+            mma_commit(&bars[B_O]);
+          }
+          mma_commit(&bars[B_EMPTY0 + st]);
+        }
+        __syncwarp();
       }
-      if (t4 == 0) CH_TS(c, 13);
+      if (lane == 0) {
+        // every MMA has completed before tensor memory is read back or released
+        mma_commit(&bars[B_DRAIN]);
+        if (!mbar_wait(&bars[B_DRAIN], 0)) fail(GDN_ERR_TIMEOUT);
+      }
     }
   }
 
@@ -658,15 +565,14 @@ __global__ void __launch_bounds__(CH_THREADS, 1) chunk_chain_kernel(
 }
 
 int g_debug_skip_chunk = -1;  // failure-test builds: chunk whose tiles the producer withholds
-unsigned long long* g_chain_trace = nullptr;  // trace builds: device buffer of 256 x 16 stamps
+unsigned long long* g_chain_trace = nullptr;  // trace builds: device buffer of 256 x 32 stamps
 
 }  // namespace
 
 cudaError_t launch_chunk_chain(const void* q, const void* k, const void* v, TokStrides ts,
                                float scale, const float* S0, const int32_t* cu, int N, int B,
                                int64_t T, int Hk, int Hv, void* out, float* S_T, void* ws,
-                               int phase, int64_t lseg, int* status, cudaStream_t s,
-                               const ChunkFusion& fuse) {
+                               int phase, int64_t lseg, int* status, cudaStream_t s) {
   const int64_t n_tok = (int64_t)B * T;
   const int64_t msegs = tm::max_segs(N, n_tok, lseg);  // lseg: the smallest the planner may pick
   // units per v-head: phase 0 one per sequence; phase 1 at most one per sequence and two per
@@ -702,9 +608,6 @@ cudaError_t launch_chunk_chain(const void* q, const void* k, const void* v, TokS
                     : reinterpret_cast<float*>(wsb + tm::states_offset(N, n_tok, Hv));
   p.debug_skip_chunk = g_debug_skip_chunk;
   p.trace = g_chain_trace;
-  p.z = fuse.z;
-  p.norm_w = fuse.norm_w;
-  p.norm_eps = fuse.norm_eps;
   static bool attr_set = false;  // idempotent attribute; a benign race between host threads
   if (!attr_set) {
     cudaError_t e = cudaFuncSetAttribute(chunk_chain_kernel,
@@ -719,7 +622,7 @@ cudaError_t launch_chunk_chain(const void* q, const void* k, const void* v, TokS
 }  // namespace gdn
 
 #ifdef GDN_CHAIN_TRACE
-// Trace builds only: device buffer (256 chunks x 16 slots of 8 bytes) for the phase stamps of CTA 0.
+// Trace builds only: device buffer (256 chunks x 32 slots of 8 bytes) for the phase stamps of CTA 0.
 extern "C" void gdn_debug_set_chain_trace(void* buf) {
   gdn::g_chain_trace = reinterpret_cast<unsigned long long*>(buf);
 }

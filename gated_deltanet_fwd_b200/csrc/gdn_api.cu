@@ -50,16 +50,16 @@ bool run_two_kernel(const void* q, const void* k, const void* v, TokStrides ts, 
       e = launch_chunk_prep(q, k, ts, g, beta, cu, N, B, T, Hk, Hv, ws, status, s, fuse);
     if (e == cudaSuccess)
       e = launch_chunk_chain(q, k, v, ts, scale, S0, cu, N, B, T, Hk, Hv, out, S_T, ws, 1, lseg,
-                             status, s, fuse);
+                             status, s);
     if (e == cudaSuccess) e = launch_scan_prefix(cu, N, B, T, Hv, lseg, ws, status, s);
     if (e == cudaSuccess)
       e = launch_chunk_chain(q, k, v, ts, scale, S0, cu, N, B, T, Hk, Hv, out, S_T, ws, 3, lseg,
-                             status, s, fuse);
+                             status, s);
   } else if (ws_bytes >= gdn::tm::workspace_bytes(N, n_tok, Hv)) {
     e = launch_chunk_prep(q, k, ts, g, beta, cu, N, B, T, Hk, Hv, ws, status, s, fuse);
     if (e == cudaSuccess)
       e = launch_chunk_chain(q, k, v, ts, scale, S0, cu, N, B, T, Hk, Hv, out, S_T, ws, 0, 0,
-                             status, s, fuse);
+                             status, s);
   } else {
     return false;
   }
@@ -281,13 +281,13 @@ gdn_status gdn_chunk_fwd_gated_norm(const void* q, int64_t q_tok_stride, const v
   fuse.b = reinterpret_cast<const __nv_bfloat16*>(b);
   fuse.A_log = A_log;
   fuse.dt_bias = dt_bias;
-  fuse.z = reinterpret_cast<const __nv_bfloat16*>(z);
-  fuse.norm_w = norm_w;
-  fuse.norm_eps = norm_eps;
   const TokStrides ts{q_tok_stride, k_tok_stride, v_tok_stride};
   cudaError_t e = cudaSuccess;
+  // the delta-rule output goes to y, and the gated RMSNorm runs over it in place
   run_two_kernel(q, k, v, ts, nullptr, nullptr, scale, initial_state, cu_seqlens, N, B, T, Hk,
                  Hv, y, final_state, workspace, workspace_bytes, status, s, fuse, &e);
+  if (e == cudaSuccess && n_tok > 0)
+    e = launch_rmsnorm(y, z, GDN_BF16, norm_w, norm_eps, n_tok * Hv, dv, y, s);
   return from_cuda(e);
 }
 

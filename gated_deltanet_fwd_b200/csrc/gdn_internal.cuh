@@ -178,9 +178,6 @@ struct ChunkFusion {
   const __nv_bfloat16* b = nullptr;
   const float* A_log = nullptr;
   const float* dt_bias = nullptr;
-  const __nv_bfloat16* z = nullptr;  // [tokens, Hv, dv] (fused gated RMSNorm when set)
-  const float* norm_w = nullptr;
-  float norm_eps = 0.0f;
 };
 
 // TMA tensor maps (tma_maps.cu), 128-byte swizzle, bf16:
@@ -201,8 +198,7 @@ cudaError_t launch_chunk_prep(const void* q, const void* k, TokStrides ts, const
 cudaError_t launch_chunk_chain(const void* q, const void* k, const void* v, TokStrides ts,
                                float scale, const float* S0, const int32_t* cu, int N, int B,
                                int64_t T, int Hk, int Hv, void* out, float* S_T, void* ws,
-                               int phase, int64_t lseg, int* status, cudaStream_t s,
-                               const ChunkFusion& fuse = ChunkFusion());
+                               int phase, int64_t lseg, int* status, cudaStream_t s);
 // One-thread planner: writes the call's segment length (0, lseg, 2 lseg or 4 lseg) into the
 // workspace for the two chain phases and the prefix to read.
 cudaError_t launch_scan_plan(const int32_t* cu, int N, int B, int64_t T, int Hv, int sms,

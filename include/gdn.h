@@ -153,9 +153,9 @@ gdn_status gdn_chunk_fwd_strided(const void* q, int64_t q_tok_stride, const void
  * gated delta rule and the gated RMSNorm of its output, as in [P3]'s flowchart (split -> gates ->
  * delta rule -> RMSNormGated(core_attn_out, z)) and [P2] §3.2.  Results equal
  *     gdn_gates(a, b) -> gdn_chunk_fwd_strided(q, k, v, g, beta) -> gdn_gated_rmsnorm(., z)
- * except that g, beta and the delta-rule output o are never written to memory: the gates are
- * computed where the per-chunk operands are prepared, and the norm is applied to the fp32 o before
- * it is rounded to bf16 (the unfused composition normalises the bf16-rounded o).
+ * except that g and beta are never written to memory: the gates are computed where the
+ * per-chunk operands are prepared.  The delta-rule output is written to y and normalised there in
+ * place by a second pass.
  * q, k, v, strides, scale, initial_state, cu_seqlens, N, B, T, Hk, Hv, final_state, workspace:
  *                  as gdn_chunk_fwd_strided.
  * a, b           : [B*T, Hv] bf16 gate pre-activations (as gdn_gates).

@@ -88,8 +88,7 @@ def test_fused_layer_core_parity(case):
                   max_abs=max_abs(y, y_ref))
     assert r <= BF16_REL_L2
     assert_bf16_close(S, S_ref, f"fused layer core state {case}")
-    # the same three steps as separate calls: the only difference is the bf16 rounding of the
-    # delta-rule output before the norm
+    # the same three steps as separate calls: they differ only in where the gates are evaluated
     y_u, S_u = _unfused(x, scale)
     assert rel_l2(y, y_u) <= BF16_REL_L2
     assert rel_l2(S, S_u) <= 1e-5
