@@ -47,12 +47,11 @@ static_assert(PP_SMEM <= 115 * 1024, "two prep CTAs per SM");
 constexpr float kLog2e = 1.4426950408889634f;
 
 // Optional phase timing, compiled in only with -DGDN_PREP_TRACE: globaltimer stamps (ns) of every
-// CTA, 8 slots per CTA, written to PrepParams::trace.
+// work item, 8 slots per item, written to PrepParams::trace.
 #ifdef GDN_PREP_TRACE
-#define PP_TS(k)                                                                       \
-  do {                                                                                 \
-    if (P.trace && tid == 0)                                                           \
-      P.trace[((size_t)blockIdx.y * gridDim.x + blockIdx.x) * 8 + (k)] = globaltimer_ns(); \
+#define PP_TS(k)                                                                   \
+  do {                                                                             \
+    if (P.trace && tid == 0) P.trace[(size_t)cur.it * 8 + (k)] = globaltimer_ns(); \
   } while (0)
 #else
 #define PP_TS(k) \
@@ -187,44 +186,72 @@ __global__ void __launch_bounds__(PP_THREADS, 2) chunk_prep_kernel(const PrepPar
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + PP_BAR + 8);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int64_t slot = blockIdx.x;
-  const int hk = blockIdx.y;
   const int G = P.Hv / P.Hk;
 
-  // ---- which chunk of which sequence this slot is (uniform across the CTA)
-  int n = -1;
-  int64_t s_beg = 0, s_end = 0, t0 = 0;
-  if (!P.cu) {
-    const int64_t per = (P.T + tm::C - 1) / tm::C;
-    if (per > 0 && slot < per * P.N) {
-      n = (int)(slot / per);
-      s_beg = (int64_t)n * P.T;
-      s_end = s_beg + P.T;
-      t0 = s_beg + (slot - (int64_t)n * per) * tm::C;
-    }
-  } else {
-    int64_t base = 0;
-    for (int m = 0; m < P.N; ++m) {
-      const int64_t a = P.cu[m], b = P.cu[m + 1];
-      if (a < 0 || b < a || b > P.T) {
-        if (tid == 0) report(P.status, GDN_ERR_DEVICE_ARG);
-        return;
+  // ---- work items (slot, k-head), item = slot * Hk + hk, strided over the persistent CTAs
+  struct Item {
+    int64_t it, slot, t0, s_end;
+    int hk, L;
+  };
+  // 1: `I` is a chunk; 0: past the last chunk (so is every later item); -1: malformed cu_seqlens
+  // (reported; nothing may be read through it).  Uniform across the CTA.
+  auto locate = [&](int64_t it, Item& I) -> int {
+    I.it = it;
+    I.slot = it / P.Hk;
+    I.hk = (int)(it - I.slot * P.Hk);
+    int n = -1;
+    int64_t s_beg = 0;
+    if (!P.cu) {
+      const int64_t per = (P.T + tm::C - 1) / tm::C;
+      if (per > 0 && I.slot < per * P.N) {
+        n = (int)(I.slot / per);
+        s_beg = (int64_t)n * P.T;
+        I.s_end = s_beg + P.T;
+        I.t0 = s_beg + (I.slot - (int64_t)n * per) * tm::C;
       }
-      const int64_t nch = (b - a + tm::C - 1) / tm::C;
-      if (slot < base + nch) {
-        n = m;
-        s_beg = a;
-        s_end = b;
-        t0 = a + (slot - base) * tm::C;
-        break;
+    } else {
+      int64_t base = 0;
+      for (int m = 0; m < P.N; ++m) {
+        const int64_t a = P.cu[m], b = P.cu[m + 1];
+        if (a < 0 || b < a || b > P.T) {
+          if (tid == 0) report(P.status, GDN_ERR_DEVICE_ARG);
+          return -1;
+        }
+        const int64_t nch = (b - a + tm::C - 1) / tm::C;
+        if (I.slot < base + nch) {
+          n = m;
+          I.s_end = b;
+          I.t0 = a + (I.slot - base) * tm::C;
+          break;
+        }
+        base += nch;
       }
-      base += nch;
     }
-  }
-  if (n < 0) return;  // slot past the last chunk
-  const int L = (int)min((int64_t)tm::C, s_end - t0);
-  PP_TS(0);
+    if (n < 0) return 0;
+    I.L = (int)min((int64_t)tm::C, I.s_end - I.t0);
+    return 1;
+  };
+  // K and Q of an item into the 128-byte-swizzled [K; Q] operand, rows >= L zero-filled:
+  // asynchronous per-thread copies (cp.async), waited for before the item's MMA
+  auto issue_loads = [&](const Item& I) {
+    constexpr int PER = 2 * 64 * 16 / PP_THREADS;
+#pragma unroll
+    for (int i = 0; i < PER; ++i) {
+      const int e = tid + i * PP_THREADS;
+      const int which = e >> 10, r = (e >> 4) & 63, ch = e & 15;
+      const int half = ch >> 3, c8 = ch & 7;
+      const __nv_bfloat16* src = (which ? P.q + (I.t0 + (r < I.L ? r : 0)) * P.q_stride
+                                        : P.k + (I.t0 + (r < I.L ? r : 0)) * P.k_stride) +
+                                 I.hk * tm::D + ch * 8;
+      cp_async16_zfill(smem + PP_KQ + half * 16384 + which * 8192 + sw128(r, c8 * 8), src,
+                       r < I.L ? 16u : 0u);
+    }
+  };
 
+  Item cur;
+  int st = locate(blockIdx.x, cur);
+  if (st <= 0) return;  // nothing allocated yet
+  PP_TS(0);
   if (tid == 0) {
     mbar_init(bar, 1);
     fence_barrier_init();
@@ -233,53 +260,45 @@ __global__ void __launch_bounds__(PP_THREADS, 2) chunk_prep_kernel(const PrepPar
     tmem_alloc(tmem_slot, 64);
     tmem_relinquish();
   }
-  // ---- K and Q of the chunk into the 128-byte-swizzled [K; Q] operand (rows >= L zero); all eight
-  // 16-byte loads of a thread are in flight before the first store
-  {
-    constexpr int PER = 2 * 64 * 16 / PP_THREADS;
-    uint4 v[PER];
+  issue_loads(cur);
+  // Once this thread's copies have landed: every thread's copies visible to the tensor core, then
+  // D1 = [K; Q] K^T of the item in shared memory (rows 0..63 K K^T, rows 64..127 Q K^T; M = 128,
+  // N = 64, K-dim 128) into tensor memory, completion signalled on `bar`.
+  auto loads_then_mma = [&](uint32_t tmem) {
+    cp_async_wait_all();
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (tid == 0) {
+      const uint32_t id = idesc_bf16(128, 64, 0, 0);
+      const uint64_t d0 = sdesc_sw128(sbase + PP_KQ, 16, 1024);
 #pragma unroll
-    for (int i = 0; i < PER; ++i) {
-      const int e = tid + i * PP_THREADS;
-      const int which = e >> 10, r = (e >> 4) & 63, ch = e & 15;
-      v[i] = make_uint4(0, 0, 0, 0);
-      if (r < L) {
-        const __nv_bfloat16* src =
-            which ? P.q + (t0 + r) * P.q_stride : P.k + (t0 + r) * P.k_stride;
-        v[i] = __ldg(reinterpret_cast<const uint4*>(src + hk * tm::D + ch * 8));
+      for (int ks = 0; ks < 8; ++ks) {
+        const uint64_t d = d0 + (uint64_t)(((ks >> 2) * 16384 + (ks & 3) * 32) >> 4);
+        mma_bf16_ss(tmem, d, d, id, ks > 0);
       }
+      mma_commit(bar);
     }
-#pragma unroll
-    for (int i = 0; i < PER; ++i) {
-      const int e = tid + i * PP_THREADS;
-      const int which = e >> 10, r = (e >> 4) & 63, ch = e & 15;
-      const int half = ch >> 3, c8 = ch & 7;
-      *reinterpret_cast<uint4*>(smem + PP_KQ + half * 16384 + which * 8192 + sw128(r, c8 * 8)) =
-          v[i];
-    }
-  }
-  fence_proxy_async_smem();
+  };
+  // the tensor-memory address is visible after the barrier in the first call
+  cp_async_wait_all();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  PP_TS(1);
   const uint32_t tmem = *tmem_slot;
-  if (tid == 0) {
-    // D1 = [K; Q] K^T: rows 0..63 K K^T, rows 64..127 Q K^T (M = 128, N = 64, K-dim 128)
-    const uint32_t id = idesc_bf16(128, 64, 0, 0);
-    const uint64_t d0 = sdesc_sw128(sbase + PP_KQ, 16, 1024);
-#pragma unroll
-    for (int ks = 0; ks < 8; ++ks) {
-      const uint64_t d = d0 + (uint64_t)(((ks >> 2) * 16384 + (ks & 3) * 32) >> 4);
-      mma_bf16_ss(tmem, d, d, id, ks > 0);
-    }
-    mma_commit(bar);
-  }
-
-  float* gl2_all = reinterpret_cast<float*>(smem + PP_GB);
-  const float* gxp = P.g;
-  const float* bxp = P.beta;
+  loads_then_mma(tmem);
+  PP_TS(1);
+  uint32_t mma_phase = 0;
   bool ok = true;
+  while (st > 0 && ok) {
+    const int64_t slot = cur.slot, t0 = cur.t0;
+    const int hk = cur.hk, L = cur.L;
+    Item nxt;
+    const int nst = locate(cur.it + gridDim.x, nxt);
+    float* gl2_all = reinterpret_cast<float*>(smem + PP_GB);
+    const float* gxp = P.g;
+    const float* bxp = P.beta;
   for (int h0 = 0; h0 < G; h0 += PAIR) {
     const int npair = min(PAIR, G - h0);
     // ---- cumulative log-decays (x log2 e) and betas of the pair's v-heads (warp gi: head gi)
@@ -324,12 +343,15 @@ __global__ void __launch_bounds__(PP_THREADS, 2) chunk_prep_kernel(const PrepPar
       gl2[96 + lane] = b1;
     }
     if (h0 == 0) {
-      ok = mbar_wait(bar, 0);
+      ok = mbar_wait(bar, mma_phase);
+      mma_phase ^= 1;
       if (!ok) report(P.status, GDN_ERR_TIMEOUT);
     }
     tc_fence_before();
     if (!__syncthreads_and(ok)) break;
     tc_fence_after();
+    // the MMA has read [K; Q]: the next item's K and Q may land there while this one is worked on
+    if (h0 == 0 && nst > 0) issue_loads(nxt);
     PP_TS(2);
     // ---- decay masks straight out of tensor memory.  Thread: row R = 32 (warp & 3) + lane of
     // [K; Q], columns 32 (warp >> 2) .. + 31.  Rows 0..63 -> A (fp32, smem), 64..127 -> P (bf16,
@@ -376,6 +398,8 @@ __global__ void __launch_bounds__(PP_THREADS, 2) chunk_prep_kernel(const PrepPar
       }
     }
     __syncthreads();  // A of every head of the pair complete
+    // after the last pair's masks D1 is free: the next item's MMA runs during this item's solve
+    if (h0 + PAIR >= G && nst > 0) loads_then_mma(tmem);
     PP_TS(3);
     // ---- T = (I + A)^{-1}: warpgroup gi solves head gi
     const int gi = warp >> 2, w4 = warp & 3, t4 = tid & 127;
@@ -413,13 +437,16 @@ __global__ void __launch_bounds__(PP_THREADS, 2) chunk_prep_kernel(const PrepPar
     __syncthreads();  // gates / A / T buffers free for the next pair
     PP_TS(5);
   }
+    cur = nxt;
+    st = nst;
+  }
+  cp_async_wait_all();  // nothing lands in shared memory after the CTA ends
   tc_fence_before();
   __syncthreads();
   if (warp == 0) {
     tc_fence_after();
     tmem_dealloc(tmem, 64);
   }
-  PP_TS(6);
 }
 
 }  // namespace
@@ -433,7 +460,7 @@ cudaError_t launch_chunk_prep(const void* q, const void* k, TokStrides ts, const
   const int64_t n_tok = (int64_t)B * T;
   const int64_t slots = tm::max_slots(N, n_tok);
   if (slots <= 0 || n_tok == 0) return cudaSuccess;
-  if (slots > 0x7fffffff || Hk > 65535) return cudaErrorInvalidConfiguration;
+  if (slots > 0x7fffffff / 64) return cudaErrorInvalidConfiguration;
   PrepParams p;
   p.q = reinterpret_cast<const __nv_bfloat16*>(q);
   p.k = reinterpret_cast<const __nv_bfloat16*>(k);
@@ -455,6 +482,7 @@ cudaError_t launch_chunk_prep(const void* q, const void* k, TokStrides ts, const
   p.A_log = fuse.A_log;
   p.dt_bias = fuse.dt_bias;
   static bool attr_set = false;  // idempotent attribute; a benign race between host threads
+  static int sms = 0;
   if (!attr_set) {
     cudaError_t e = cudaFuncSetAttribute(chunk_prep_kernel,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, PP_SMEM);
@@ -462,10 +490,16 @@ cudaError_t launch_chunk_prep(const void* q, const void* k, TokStrides ts, const
     if (e == cudaSuccess)
       e = cudaFuncSetAttribute(chunk_prep_kernel,
                                cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+    int dev = 0;
+    if (e == cudaSuccess) e = cudaGetDevice(&dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  chunk_prep_kernel<<<dim3((unsigned)slots, (unsigned)Hk), PP_THREADS, PP_SMEM, s>>>(p);
+  // persistent: two CTAs per SM, each taking every grid-th (slot, k-head) item
+  const int64_t items = slots * Hk;
+  const int64_t grid = items < 2 * (int64_t)sms ? items : 2 * (int64_t)sms;
+  chunk_prep_kernel<<<(unsigned)grid, PP_THREADS, PP_SMEM, s>>>(p);
   return cudaGetLastError();
 }
 

@@ -146,6 +146,19 @@ __device__ __forceinline__ void bulk_wait() {
   asm volatile("cp.async.bulk.wait_group %0;" ::"n"(N) : "memory");
 }
 
+// Per-thread 16-byte global -> shared copy that reads `src_bytes` (16 or 0) bytes and zero-fills
+// the rest; the thread sees its own copies after cp_async_wait_all().
+__device__ __forceinline__ void cp_async16_zfill(void* smem_dst, const void* gsrc,
+                                                 uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(smem_dst)),
+               "l"(gsrc), "r"(src_bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.commit_group;\ncp.async.wait_group 0;" ::: "memory");
+}
+
 // ------------------------------------------------------------------ tcgen05 ----------------
 // Tensor memory: 128 lanes x 512 columns of 32 bits per SM.  A TMEM address is (lane << 16) | col.
 
