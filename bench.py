@@ -52,23 +52,36 @@ CHUNK_LAUNCHES = 5
 # capture each (summaries under profiles/), tied to the kernel source they were taken from: once
 # the source changes the bench reports traffic as null until it is captured again.
 MEASURED_TRAFFIC = {
-    # chunk_tc_kernel on B=1, T=4096 (prefill 4K): 68.2 MB read + 8.8 MB written = 18,805 B per
-    # token over all 32 heads; scaled by the tokens of a launch (reads scale with tokens; the
-    # write count is a lower bound, the output drains from L2 after the kernel).
-    "gdn_chunk_fwd": dict(source="csrc/chunk_tc.cu", sha256_16="d91b1956d8eb683c",
-                          bytes_per_token=77027072 / 4096),
+    # one gdn_chunk_fwd call on the 32K varlen workload (scan plan, prep, chain phase 1, state
+    # prefix, chain phase 3), ncu dram__bytes_read.sum + dram__bytes_write.sum summed over the
+    # five kernels: 1,390.9 MB read + 462.1 MB written (profiles/chunk_prefill_varlen_32k_dram.md)
+    "gdn_chunk_fwd": dict(sources=["csrc/chunk_prep.cu", "csrc/chunk_chain.cu",
+                                   "csrc/chunk_scan.cu", "csrc/chunk_tm.cuh"],
+                          sha256_16="7ca324b8739785dd", bytes_per_launch=1.85296e9),
     # recurrent_step_kernel on 256 sequences x 32 heads: 5.92 TB/s x 172.8 us.
-    "gdn_recurrent_step": dict(source="csrc/recurrent.cu", sha256_16="b07ec22be73c2392",
+    "gdn_recurrent_step": dict(sources=["csrc/recurrent.cu"], sha256_16="b07ec22be73c2392",
                                bytes_per_launch=1.0224e9),
+    # decode_fused_kernel on 256 sequences x 32 heads: 568.6 MB read + 507.5 MB written
+    # (profiles/decode_fused_decode_layer_256.md)
+    "gdn_decode_layer_step": dict(sources=["csrc/decode_fused.cu"], sha256_16="5cccc0f4eda2ae9c",
+                                  bytes_per_launch=1.07607e9),
 }
 
 
+def _sources_sha(sources):
+    h = hashlib.sha256()
+    for src in sources:
+        with open(os.path.join(ROOT, "gated_deltanet_fwd_b200", src), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
 def _traffic(kernel, units):
+    """ncu DRAM bytes per launch of `kernel` scaled to `units`, or None once a source it was
+    measured on has changed."""
     m = MEASURED_TRAFFIC[kernel]
-    path = os.path.join(ROOT, "gated_deltanet_fwd_b200", m["source"])
     try:
-        with open(path, "rb") as f:
-            sha = hashlib.sha256(f.read()).hexdigest()[:16]
+        sha = _sources_sha(m["sources"])
     except OSError:
         return None
     if sha != m["sha256_16"]:
@@ -402,6 +415,8 @@ def bench_decode_layer(dist, gdn, K, W, peaks):
                 roofline=dict(bound="hbm", kernel="gdn_decode_layer_step", achieved=achieved,
                               peak=peaks["hbm"], unit="GB/s", frac=achieved / peaks["hbm"],
                               frac_of_nominal_8tbs=achieved / 8000.0,
+                              traffic=_traffic("gdn_decode_layer_step", 1),
+                              traffic_unit="bytes per launch",
                               bytes_per_launch=bytes_per_launch,
                               peak_source=peaks["source"] + " HBM copy"),
                 gpu_launches=steps * K)
@@ -473,7 +488,7 @@ def bench_layer_core(dist, gdn, K, W, peaks):
                 conv_hbm_frac=conv_bytes / (per["conv"] * 1e-3) / 1e9 / peaks["hbm"],
                 core_tensor_frac=flop / (per["core"] * 1e-3) / 1e12 / peaks["bf16"],
                 unfused=dict(ms_per_step=ms_u / K, kernels_ms=per_u),
-                gpu_launches=(1 + CHUNK_LAUNCHES) * K)
+                gpu_launches=(1 + CHUNK_LAUNCHES + 1) * K)
 
 
 # ------------------------------------------------------------------ CPU oracle --------------
@@ -539,6 +554,7 @@ def run_profile(mode, reps):
                v channels viewed as 128-wide rows
     layercore  the layer core on B = 2 x 16384 tokens: gdn_causal_conv1d_silu, then
                gdn_chunk_fwd_gated_norm on q, k, v read in place from the conv output
+    decodelayer  consecutive gdn_decode_layer_step calls on 256 sequences x 32 heads
     """
     from gated_deltanet_fwd_b200 import gdn
     dev = torch.device("cuda", 0)
@@ -569,6 +585,17 @@ def run_profile(mode, reps):
         for _ in range(reps):
             y = gdn.gdn_causal_conv1d_silu(mix, cw, None, n_l2norm_ch=nqk, l2norm_group=w["dk"])
             gdn.gdn_gated_rmsnorm(y[:, :, nqk:].contiguous().view(-1, w["dv"]), z, nw)
+    elif mode == "decodelayer":
+        w = dict(inputs.WORKLOADS["decode_layer_256"], steps=max(reps, 1))
+        x = inputs.decode_layer_inputs(**w, seed=1000 + w["index"])
+        st = x["state"].to(dev)
+        cs = [x["conv_state"].to(dev), torch.empty_like(x["conv_state"]).to(dev)]
+        cw, A_log, dt_bias = x["conv_w"].to(dev), x["A_log"].to(dev), x["dt_bias"].to(dev)
+        nw = x["norm_w"].to(dev)
+        for s_ in range(w["steps"]):
+            gdn.gdn_decode_layer_step(x["mix"][s_].to(dev), x["a"][s_].to(dev),
+                                      x["b"][s_].to(dev), x["z"][s_].to(dev), cw, cs[s_ & 1],
+                                      cs[(s_ + 1) & 1], A_log, dt_bias, nw, st, w["Hk"])
     elif mode == "layercore":
         w = inputs.WORKLOADS["layer_core_2x16k"]
         x = inputs.layer_core_inputs(**w, seed=1000 + w["index"])
@@ -600,7 +627,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--profile", default=None,
                     help="run one workload for a profiler capture: "
-                         "prefill|prefill4k|decode|conv|layercore")
+                         "prefill|prefill4k|decode|conv|layercore|decodelayer")
     ap.add_argument("--repeats", type=int, default=2, help="launches per --profile run")
     args = ap.parse_args()
     if args.profile:
