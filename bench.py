@@ -54,7 +54,7 @@ CHUNK_LAUNCHES = 5
 MEASURED_TRAFFIC = {
     # one gdn_chunk_fwd call on the 32K varlen workload (scan plan, prep, chain phase 1, state
     # prefix, chain phase 3), ncu dram__bytes_read.sum + dram__bytes_write.sum summed over the
-    # five kernels: 1,390.9 MB read + 462.1 MB written (profiles/chunk_prefill_varlen_32k_dram.md)
+    # five kernels: 1,390.9 MB read + 462.1 MB written
     "gdn_chunk_fwd": dict(sources=["csrc/chunk_prep.cu", "csrc/chunk_chain.cu",
                                    "csrc/chunk_scan.cu", "csrc/chunk_tm.cuh"],
                           sha256_16="7ca324b8739785dd", bytes_per_launch=1.85296e9),
@@ -62,7 +62,7 @@ MEASURED_TRAFFIC = {
     "gdn_recurrent_step": dict(sources=["csrc/recurrent.cu"], sha256_16="b07ec22be73c2392",
                                bytes_per_launch=1.0224e9),
     # decode_fused_kernel on 256 sequences x 32 heads: 568.6 MB read + 507.5 MB written
-    # (profiles/decode_fused_decode_layer_256.md)
+    # (ncu, one launch)
     "gdn_decode_layer_step": dict(sources=["csrc/decode_fused.cu"], sha256_16="5cccc0f4eda2ae9c",
                                   bytes_per_launch=1.07607e9),
 }
