@@ -33,22 +33,44 @@ __device__ __forceinline__ float dwarp_sum(float x) {
   return x;
 }
 
-// silu(conv of one channel over the K-1 cached inputs and the new one); also writes the channel's
-// shifted history to cs_out when `write_state`.
+// One channel's conv inputs: the new input, its K-1 cached predecessors (oldest first) and the
+// K taps.  Loaded for all of a thread's channels before any of them is computed or its history
+// written, so that the loads form one round trip.
+struct ConvIn {
+  float xt, bias;
+  float hist[7];
+  float w[8];
+};
+
 template <typename T>
-__device__ __forceinline__ float conv_channel(const T* x, const float* w, const float* bias,
-                                             int K, int64_t c, const float* cs_in, float* cs_out,
-                                             bool write_state) {
-  const float xt = to_f(x[c]);
-  float acc = bias ? __ldg(bias + c) : 0.0f;
-  const float* wc = w + c * K;
-  const float* hin = cs_in + c * (K - 1);
-  for (int i = 0; i < K - 1; ++i) acc = fmaf(__ldg(wc + i), hin[i], acc);
-  acc = fmaf(__ldg(wc + K - 1), xt, acc);
+__device__ __forceinline__ void conv_load(ConvIn& ci, const T* __restrict__ x,
+                                          const float* __restrict__ w,
+                                          const float* __restrict__ bias, int K, int64_t c,
+                                          const float* __restrict__ cs_in) {
+  ci.xt = to_f(x[c]);
+  ci.bias = bias ? __ldg(bias + c) : 0.0f;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) ci.w[i] = i < K ? __ldg(w + c * K + i) : 0.0f;
+#pragma unroll
+  for (int i = 0; i < 7; ++i) ci.hist[i] = i < K - 1 ? cs_in[c * (K - 1) + i] : 0.0f;
+}
+
+// silu(conv) of a loaded channel; writes its history shifted by this token when `write_state`
+__device__ __forceinline__ float conv_finish(const ConvIn& ci, int K, int64_t c,
+                                             float* __restrict__ cs_out, bool write_state) {
+  float acc = ci.bias;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {  // tap i: cached input i, or the new input at i = K - 1
+    // (i < K - 1 <= 7 whenever hist is read; the clamp only keeps the index constant-foldable)
+    const float xi = i < K - 1 ? ci.hist[i < 7 ? i : 6] : (i == K - 1 ? ci.xt : 0.0f);
+    acc = fmaf(ci.w[i], xi, acc);
+  }
   if (write_state && K > 1) {
     float* hout = cs_out + c * (K - 1);
-    for (int i = 0; i + 1 < K - 1; ++i) hout[i] = hin[i + 1];
-    hout[K - 2] = xt;
+#pragma unroll
+    for (int i = 0; i < 6; ++i)
+      if (i + 1 < K - 1) hout[i] = ci.hist[i + 1];
+    hout[K - 2] = ci.xt;
   }
   return siluf_(acc);
 }
@@ -92,6 +114,13 @@ __global__ void __launch_bounds__(DF_THREADS, 3) decode_fused_kernel(const Decod
       s[u] = __ldcs(reinterpret_cast<const float4*>(Sb + u * DF_D) + lane);
   }
 
+  // the warp's second batch of rows, towards L2 (one 128-byte line per lane: row lane / 4, line
+  // lane % 4), so that its loads after the first batch are L2 hits
+  {
+    const float* Sb2 = S + (size_t)(warp * DF_ROWS + (DF_THREADS / 32) * DF_ROWS) * DF_D;
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(Sb2 + (lane >> 2) * DF_D + 32 * (lane & 3)));
+  }
+
   // the gate of the output norm, requested early as well
   const float zv = tid < DF_D ? to_f(reinterpret_cast<const T*>(P.z)[(int64_t)nh * DF_D + tid])
                               : 0.0f;
@@ -102,16 +131,14 @@ __global__ void __launch_bounds__(DF_THREADS, 3) decode_fused_kernel(const Decod
   float* cs_out = P.cs_out + (int64_t)n * P.C * (P.K - 1);
   const int j = tid & (DF_D - 1);
   const bool qk_owner = (h % G) == 0;  // one v-head per k-head advances the q/k history
-  float qk;  // q (threads < 128) or k (threads >= 128) before the norm
-  if (tid < DF_D) {
-    qk = conv_channel(x, P.conv_w, P.conv_bias, P.K, (int64_t)hk * DF_D + j, cs_in, cs_out,
-                      qk_owner);
-    v_s[j] = conv_channel(x, P.conv_w, P.conv_bias, P.K,
-                          2 * (int64_t)P.Hk * DF_D + (int64_t)h * DF_D + j, cs_in, cs_out, true);
-  } else {
-    qk = conv_channel(x, P.conv_w, P.conv_bias, P.K, (int64_t)(P.Hk + hk) * DF_D + j, cs_in,
-                      cs_out, qk_owner);
-  }
+  // threads < 128: q channel j and v channel j; threads >= 128: k channel j
+  const int64_t c_qk = tid < DF_D ? (int64_t)hk * DF_D + j : (int64_t)(P.Hk + hk) * DF_D + j;
+  const int64_t c_v = 2 * (int64_t)P.Hk * DF_D + (int64_t)h * DF_D + j;
+  ConvIn in_qk, in_v;
+  conv_load(in_qk, x, P.conv_w, P.conv_bias, P.K, c_qk, cs_in);
+  if (tid < DF_D) conv_load(in_v, x, P.conv_w, P.conv_bias, P.K, c_v, cs_in);
+  const float qk = conv_finish(in_qk, P.K, c_qk, cs_out, qk_owner);  // q or k before the norm
+  if (tid < DF_D) v_s[j] = conv_finish(in_v, P.K, c_v, cs_out, true);
   // per-head L2 norm of q (warps 0-3) and k (warps 4-7)
   const float ss = dwarp_sum(qk * qk);
   if (lane == 0) red[warp] = ss;

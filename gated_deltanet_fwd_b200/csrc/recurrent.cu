@@ -38,6 +38,15 @@ __global__ void __launch_bounds__(REC_THREADS, 3) recurrent_step_kernel(
   const int hk = h / (Hv / Hk);
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
 
+  // the warp's first two batches of state rows are requested towards L2 before the q/k/gate
+  // round trip (one 128-byte line per lane: row lane / 4 of the batch, line lane % 4)
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    const int row = warp * REC_ROWS + i * (REC_THREADS / 32) * REC_ROWS + (lane >> 2);
+    if (row < dv)
+      asm volatile("prefetch.global.L2 [%0];" ::"l"(state + ((int64_t)nh * dv + row) * DK +
+                                                      32 * (lane & 3)));
+  }
   float k4[4], q4[4];
   load4(k + ((int64_t)n * Hk + hk) * DK + 4 * lane, k4);
   load4(q + ((int64_t)n * Hk + hk) * DK + 4 * lane, q4);
