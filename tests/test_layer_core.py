@@ -78,7 +78,7 @@ def test_layer_core_end_to_end_full_size():
         o_ref, S_ref = oracle.gated_delta_rule(q_ref, k_ref, v_ref, g_ref[bi:bi + 1],
                                                b_ref[bi:bi + 1], scale, nthreads=NTHREADS)
         del q_ref, k_ref, v_ref
-        # delta-rule stage, the benchmark spec's tolerance on outputs and final state
+        # delta-rule stage, the method's bf16 tolerance on outputs and final state
         assert_bf16_close(core_gpu[bi:bi + 1], o_ref, f"layer core chunk output, row {bi}")
         assert_bf16_close(S_gpu[bi:bi + 1], S_ref, f"layer core final state, row {bi}")
         # normed output: RMSNorm rescales each row, so its error is the core output's relative
