@@ -162,6 +162,7 @@ __global__ void __launch_bounds__(DF_THREADS, 3) decode_fused_kernel(const Decod
   const float4 k4 = reinterpret_cast<const float4*>(k_s)[lane];
   const float4 q4 = reinterpret_cast<const float4*>(q_s)[lane];
   const float kq = dwarp_sum(k4.x * q4.x + k4.y * q4.y + k4.z * q4.z + k4.w * q4.w);
+  float oss = 0.0f;  // this warp's share of sum(o^2) for the norm (the same in every lane)
   for (int base = warp * DF_ROWS; base < DF_D; base += (DF_THREADS / 32) * DF_ROWS) {
     if (base != warp * DF_ROWS) {
       const float* Sb = S + (size_t)base * DF_D;
@@ -185,20 +186,19 @@ __global__ void __launch_bounds__(DF_THREADS, 3) decode_fused_kernel(const Decod
       o4.z = fmaf(a, s[u].z, uj * k4.z);
       o4.w = fmaf(a, s[u].w, uj * k4.w);
       __stcs(reinterpret_cast<float4*>(S + (size_t)r * DF_D) + lane, o4);
-      if (lane == u) o_s[r] = P.scale * fmaf(a, sq[u], uj * kq);
+      const float o = P.scale * fmaf(a, sq[u], uj * kq);  // uniform across the warp
+      oss = fmaf(o, o, oss);
+      if (lane == u) o_s[r] = o;
     }
   }
+  if (lane == 0) red[8 + warp] = oss;
   __syncthreads();
 
   // ---- gated RMSNorm of the head's output: y = o rsqrt(mean o^2 + eps) (1 + w) silu(z)
   if (tid < DF_D) {
-    const float o = o_s[tid];
-    const float so = dwarp_sum(o * o);
-    if (lane == 0) red[8 + warp] = so;
-  }
-  __syncthreads();
-  if (tid < DF_D) {
-    const float inv = rsqrtf((red[8] + red[9] + red[10] + red[11]) * (1.0f / DF_D) + P.norm_eps);
+    const float tot = ((red[8] + red[9]) + (red[10] + red[11])) +
+                      ((red[12] + red[13]) + (red[14] + red[15]));
+    const float inv = rsqrtf(tot * (1.0f / DF_D) + P.norm_eps);
     const float yv = o_s[tid] * inv * (1.0f + __ldg(P.norm_w + tid)) * siluf_(zv);
     reinterpret_cast<T*>(P.y)[(int64_t)nh * DF_D + tid] = from_f<T>(yv);
   }
