@@ -5,6 +5,8 @@
 // and never trap.
 #include <stdio.h>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "chunk_tm.cuh"
 #include "gdn_internal.cuh"
 
@@ -13,6 +15,16 @@ using namespace gdn;
 namespace {
 
 inline cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
+
+// An NVTX range named after the ABI call for the duration of its host side (argument checks and
+// launches), so that a profiler's timeline shows which call enqueued which kernels.  Without an
+// attached tool the push and pop are no-ops.
+struct CallRange {
+  explicit CallRange(const char* name) { nvtxRangePushA(name); }
+  ~CallRange() { nvtxRangePop(); }
+  CallRange(const CallRange&) = delete;
+  CallRange& operator=(const CallRange&) = delete;
+};
 
 inline bool bad_dtype(gdn_dtype d) { return d != GDN_BF16 && d != GDN_F32; }
 
@@ -92,6 +104,7 @@ const char* gdn_status_string(gdn_status s) {
 gdn_status gdn_gates(const void* a, const void* b, gdn_dtype ab_dtype, const float* A_log,
                      const float* dt_bias, int64_t n_tok, int Hv, float* g, float* beta,
                      void* stream) {
+  CallRange range_("gdn_gates");
   if (bad_dtype(ab_dtype) || n_tok < 0 || Hv < 1) return GDN_ERR_INVALID_ARG;
   if (n_tok == 0) return GDN_OK;
   if (!a || !b || !A_log || !dt_bias || !g || !beta) return GDN_ERR_INVALID_ARG;
@@ -104,6 +117,7 @@ gdn_status gdn_causal_conv1d_silu(const void* x, gdn_dtype dtype, const float* w
                                   const int32_t* cu_seqlens, int N, int n_l2norm_ch,
                                   int l2norm_group, float l2_eps, const float* conv_state_in,
                                   float* conv_state_out, void* y, void* stream) {
+  CallRange range_("gdn_causal_conv1d_silu");
   if (bad_dtype(dtype) || B < 0 || T < 0 || C < 1 || K < 1 || N < 0) return GDN_ERR_INVALID_ARG;
   if (cu_seqlens ? (B != 1 && !(B == 0 && T == 0)) : (N != B)) return GDN_ERR_INVALID_ARG;
   if (n_l2norm_ch < 0 || n_l2norm_ch > C || l2norm_group < 0) return GDN_ERR_INVALID_ARG;
@@ -177,6 +191,7 @@ gdn_status gdn_chunk_fwd_strided(const void* q, int64_t q_tok_stride, const void
                                  int B, int64_t T, int Hk, int Hv, int dk, int dv, int chunk,
                                  void* out, float* final_state, void* workspace,
                                  size_t workspace_bytes, void* stream) {
+  CallRange range_("gdn_chunk_fwd_strided");
   if (bad_dtype(dtype) || N < 0 || B < 0 || T < 0 || Hk < 1 || Hv < 1 || dk < 1 || dv < 1)
     return GDN_ERR_INVALID_ARG;
   if (Hv % Hk != 0) return GDN_ERR_INVALID_ARG;
@@ -243,6 +258,7 @@ gdn_status gdn_chunk_fwd_gated_norm(const void* q, int64_t q_tok_stride, const v
                                     int B, int64_t T, int Hk, int Hv, int dk, int dv, int chunk,
                                     void* y, float* final_state, void* workspace,
                                     size_t workspace_bytes, void* stream) {
+  CallRange range_("gdn_chunk_fwd_gated_norm");
   if (bad_dtype(dtype) || N < 0 || B < 0 || T < 0 || Hk < 1 || Hv < 1 || dk < 1 || dv < 1)
     return GDN_ERR_INVALID_ARG;
   if (Hv % Hk != 0) return GDN_ERR_INVALID_ARG;
@@ -294,6 +310,7 @@ gdn_status gdn_chunk_fwd_gated_norm(const void* q, int64_t q_tok_stride, const v
 gdn_status gdn_recurrent_step(const void* q, const void* k, const void* v, const float* g,
                               const float* beta, gdn_dtype dtype, float scale, float* state,
                               int N, int Hk, int Hv, int dk, int dv, void* out, void* stream) {
+  CallRange range_("gdn_recurrent_step");
   if (bad_dtype(dtype) || N < 0 || Hk < 1 || Hv < 1 || dk < 1 || dv < 1)
     return GDN_ERR_INVALID_ARG;
   if (Hv % Hk != 0) return GDN_ERR_INVALID_ARG;
@@ -313,6 +330,7 @@ gdn_status gdn_decode_layer_step(const void* mix, const void* a, const void* b, 
                                  const float* A_log, const float* dt_bias, const float* norm_w,
                                  float l2_eps, float norm_eps, float scale, float* state, int N,
                                  int Hk, int Hv, int dk, int dv, void* y, void* stream) {
+  CallRange range_("gdn_decode_layer_step");
   if (bad_dtype(dtype) || N < 0 || Hk < 1 || Hv < 1 || dk < 1 || dv < 1 || K < 1)
     return GDN_ERR_INVALID_ARG;
   if (Hv % Hk != 0) return GDN_ERR_INVALID_ARG;
@@ -337,6 +355,7 @@ gdn_status gdn_decode_layer_step(const void* mix, const void* a, const void* b, 
 
 gdn_status gdn_gated_rmsnorm(const void* x, const void* z, gdn_dtype dtype, const float* w,
                              float eps, int64_t n_rows, int dim, void* y, void* stream) {
+  CallRange range_("gdn_gated_rmsnorm");
   if (bad_dtype(dtype) || n_rows < 0 || dim < 1 || !(eps >= 0.0f)) return GDN_ERR_INVALID_ARG;
   if (dim != 8 && dim != 16 && dim != 32 && dim != 64 && dim != 128 && dim != 256)
     return GDN_ERR_UNSUPPORTED;
