@@ -11,7 +11,7 @@
 namespace gdn {
 namespace ptx {
 
-constexpr uint32_t kSpinLimit = 1u << 26;  // ~ seconds of polling with the suspend hint
+constexpr uint32_t kSpinLimit = 1u << 26;  // a cap on polls; the wall-clock limit normally ends a wait first
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -47,17 +47,18 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t by
                : "memory");
 }
 
-// One bounded poll.  The suspend-time hint (ns) lets the hardware park the thread until the phase
-// completes (or the hint expires) instead of spinning, so waiting warps leave the issue slots to
-// the warps that are working.
+// One bounded poll: the hardware holds the thread for a short, implementation-defined time while
+// the phase is incomplete and returns false if it stays so.  (A suspend-time hint, which parks the
+// thread until completion, measured 0.7 % slower on the prefill: the woken warps of the chunk
+// chain resume later.)
 __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity), "r"(1000000u)
+      : "r"(smem_u32(bar)), "r"(parity)
       : "memory");
   return ok != 0;
 }
