@@ -204,6 +204,115 @@ __global__ void __launch_bounds__(DF_THREADS, 3) decode_fused_kernel(const Decod
   }
 }
 
+// The same step with both v-heads of a k-head in one block (Hv = 2 Hk): the q/k conv and norms
+// are done once for the pair, and the prologue is spread over twice the state bytes.  Threads
+// 0..127 own q channel j and v channel j of the first head, threads 128..255 k channel j and v
+// channel j of the second; warps 0-3 update the first head's rows, warps 4-7 the second's, each
+// 32 rows in four batches of 8.
+template <typename T>
+__global__ void __launch_bounds__(DF_THREADS, 3) decode_fused_pair_kernel(const DecodeParams P) {
+  __shared__ float q_s[DF_D], k_s[DF_D], v_s[2][DF_D], o_s[2][DF_D];
+  __shared__ float red[16];
+  __shared__ float gate_s[2][2];
+  const int nk = blockIdx.x;  // n * Hk + hk
+  const int n = nk / P.Hk, hk = nk - n * P.Hk;
+  const int64_t nh0 = (int64_t)n * P.Hv + 2 * hk;  // the pair's first v-head (n, 2 hk)
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int hw = warp >> 2;  // the head whose rows this warp updates
+  float* S = P.state + (nh0 + hw) * DF_D * DF_D;
+  constexpr int kBatches = DF_D / (4 * DF_ROWS);  // 4 batches of 8 rows per warp
+  const int row0 = DF_ROWS * (warp & 3);           // batch b: rows row0 + 32 b .. + 7
+
+  // ---- the first batch of rows in flight before the prologue, the others towards L2
+  float4 s[DF_ROWS];
+#pragma unroll
+  for (int u = 0; u < DF_ROWS; ++u)
+    s[u] = __ldcs(reinterpret_cast<const float4*>(S + (size_t)(row0 + u) * DF_D) + lane);
+#pragma unroll
+  for (int b = 1; b < kBatches; ++b)
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(S + (size_t)(row0 + 32 * b + (lane >> 2)) * DF_D +
+                                                  32 * (lane & 3)));
+  // z of both heads (contiguous)
+  const float zv = to_f(reinterpret_cast<const T*>(P.z)[nh0 * DF_D + tid]);
+
+  // ---- conv + SiLU
+  const T* x = reinterpret_cast<const T*>(P.mix) + (int64_t)n * P.C;
+  const float* cs_in = P.cs_in + (int64_t)n * P.C * (P.K - 1);
+  float* cs_out = P.cs_out + (int64_t)n * P.C * (P.K - 1);
+  const int j = tid & (DF_D - 1), hv = tid >> 7;
+  const int64_t c_qk = hv == 0 ? (int64_t)hk * DF_D + j : (int64_t)(P.Hk + hk) * DF_D + j;
+  const int64_t c_v = 2 * (int64_t)P.Hk * DF_D + (2 * hk + hv) * (int64_t)DF_D + j;
+  ConvIn in_qk, in_v;
+  conv_load(in_qk, x, P.conv_w, P.conv_bias, P.K, c_qk, cs_in);
+  conv_load(in_v, x, P.conv_w, P.conv_bias, P.K, c_v, cs_in);
+  const float qk = conv_finish(in_qk, P.K, c_qk, cs_out, true);  // q or k before the norm
+  v_s[hv][j] = conv_finish(in_v, P.K, c_v, cs_out, true);
+  const float ss = dwarp_sum(qk * qk);
+  if (lane == 0) red[warp] = ss;
+  if (j == 0) {  // threads 0 and 128: the gates of their head
+    const int h = 2 * hk + hv;
+    const float av = to_f(reinterpret_cast<const T*>(P.a)[nh0 + hv]);
+    const float bv = to_f(reinterpret_cast<const T*>(P.b)[nh0 + hv]);
+    gate_s[hv][0] = sigmoidf_(bv);
+    gate_s[hv][1] = expf(-expf(__ldg(P.A_log + h)) * softplusf_(av + __ldg(P.dt_bias + h)));
+  }
+  __syncthreads();
+  {
+    const int g0 = hv == 0 ? 0 : 4;
+    const float tot = red[g0] + red[g0 + 1] + red[g0 + 2] + red[g0 + 3];
+    const float inv = rsqrtf(tot + P.l2_eps);
+    if (hv == 0) q_s[j] = qk * inv; else k_s[j] = qk * inv;
+  }
+  __syncthreads();
+
+  // ---- the recurrent step of this warp's head, four batches of 8 rows
+  const float b = gate_s[hw][0], a = gate_s[hw][1];
+  const float4 k4 = reinterpret_cast<const float4*>(k_s)[lane];
+  const float4 q4 = reinterpret_cast<const float4*>(q_s)[lane];
+  const float kq = dwarp_sum(k4.x * q4.x + k4.y * q4.y + k4.z * q4.z + k4.w * q4.w);
+  float oss = 0.0f;
+#pragma unroll 1
+  for (int bt = 0; bt < kBatches; ++bt) {
+    const int base = row0 + 32 * bt;
+    if (bt > 0) {
+#pragma unroll
+      for (int u = 0; u < DF_ROWS; ++u)
+        s[u] = __ldcs(reinterpret_cast<const float4*>(S + (size_t)(base + u) * DF_D) + lane);
+    }
+    float sk[DF_ROWS], sq[DF_ROWS];
+#pragma unroll
+    for (int u = 0; u < DF_ROWS; ++u) {
+      sk[u] = dwarp_sum(s[u].x * k4.x + s[u].y * k4.y + s[u].z * k4.z + s[u].w * k4.w);
+      sq[u] = dwarp_sum(s[u].x * q4.x + s[u].y * q4.y + s[u].z * q4.z + s[u].w * q4.w);
+    }
+#pragma unroll
+    for (int u = 0; u < DF_ROWS; ++u) {
+      const int r = base + u;
+      const float uj = b * (v_s[hw][r] - a * sk[u]);
+      float4 o4;
+      o4.x = fmaf(a, s[u].x, uj * k4.x);
+      o4.y = fmaf(a, s[u].y, uj * k4.y);
+      o4.z = fmaf(a, s[u].z, uj * k4.z);
+      o4.w = fmaf(a, s[u].w, uj * k4.w);
+      __stcs(reinterpret_cast<float4*>(S + (size_t)r * DF_D) + lane, o4);
+      const float o = P.scale * fmaf(a, sq[u], uj * kq);  // uniform across the warp
+      oss = fmaf(o, o, oss);
+      if (lane == u) o_s[hw][r] = o;
+    }
+  }
+  if (lane == 0) red[8 + warp] = oss;
+  __syncthreads();
+
+  // ---- gated RMSNorm of each head's output (thread: head hv, column j)
+  {
+    const int r0 = 8 + 4 * hv;
+    const float tot = (red[r0] + red[r0 + 1]) + (red[r0 + 2] + red[r0 + 3]);
+    const float inv = rsqrtf(tot * (1.0f / DF_D) + P.norm_eps);
+    const float yv = o_s[hv][j] * inv * (1.0f + __ldg(P.norm_w + j)) * siluf_(zv);
+    reinterpret_cast<T*>(P.y)[nh0 * DF_D + tid] = from_f<T>(yv);
+  }
+}
+
 }  // namespace
 
 cudaError_t launch_decode_fused(const void* mix, const void* a, const void* b, const void* z,
@@ -236,10 +345,17 @@ cudaError_t launch_decode_fused(const void* mix, const void* a, const void* b, c
   p.Hk = Hk;
   p.Hv = Hv;
   p.C = 2 * (int64_t)Hk * DF_D + (int64_t)Hv * DF_D;
-  if (dt == GDN_BF16)
+  if (Hv == 2 * Hk) {  // both v-heads of a k-head in one block
+    const unsigned pairs = (unsigned)(blocks / 2);
+    if (dt == GDN_BF16)
+      decode_fused_pair_kernel<__nv_bfloat16><<<pairs, DF_THREADS, 0, s>>>(p);
+    else
+      decode_fused_pair_kernel<float><<<pairs, DF_THREADS, 0, s>>>(p);
+  } else if (dt == GDN_BF16) {
     decode_fused_kernel<__nv_bfloat16><<<(unsigned)blocks, DF_THREADS, 0, s>>>(p);
-  else
+  } else {
     decode_fused_kernel<float><<<(unsigned)blocks, DF_THREADS, 0, s>>>(p);
+  }
   return cudaGetLastError();
 }
 

@@ -77,6 +77,15 @@ def test_decode_layer_small(dtype, K):
     _run(d, 2, 128, 3, dtype, K)
 
 
+@pytest.mark.parametrize("Hk,Hv", [(2, 2), (1, 4), (3, 6)])
+def test_decode_layer_head_sharing(Hk, Hv):
+    """Other head-sharing ratios than the workload's Hv = 2 Hk (which takes the paired-head
+    kernel): one v-head per k-head, four per k-head, and three pairs."""
+    d = inputs.decode_layer_inputs(N=3, Hk=Hk, Hv=Hv, dk=128, dv=128, K=4, dtype="bf16",
+                                   seed=40 + Hk + Hv, steps=2)
+    _run(d, Hk, 128, 2, "bf16", 4)
+
+
 def test_decode_layer_full_size():
     """256 sequences, 16 q/k heads, 32 v heads, conv kernel 4, 64 consecutive tokens: every
     output of every step, every history and every final state."""
