@@ -61,9 +61,9 @@ MEASURED_TRAFFIC = {
     # recurrent_step_kernel on 256 sequences x 32 heads: 541.2 MB read + 479.2 MB written
     "gdn_recurrent_step": dict(sources=["csrc/recurrent.cu"], sha256_16="a413ca6c4c9f6c5e",
                                bytes_per_launch=1.02039e9),
-    # decode_fused_kernel on 256 sequences x 32 heads: 568.6 MB read + 507.6 MB written
-    "gdn_decode_layer_step": dict(sources=["csrc/decode_fused.cu"], sha256_16="3a5cfd9008515bec",
-                                  bytes_per_launch=1.07618e9),
+    # decode_fused_pair_kernel on 256 sequences x 32 heads: 574.8 MB read + 505.3 MB written
+    "gdn_decode_layer_step": dict(sources=["csrc/decode_fused.cu"], sha256_16="9cc12723f08fc19a",
+                                  bytes_per_launch=1.08017e9),
 }
 
 
