@@ -1,6 +1,7 @@
 // chunk_chain.cu -- the state-carrying half of the tensor-core prefill (bf16, dk = dv = 128,
-// chunks of 64 tokens): one CTA per (sequence, v-head) walks the chunks in order with the fp32
-// state held in tensor memory.
+// chunks of 64 tokens): one CTA per unit -- a whole sequence, or one segment of it under the
+// intra-sequence scan (chunk_tm.cuh), for one v-head -- walks the unit's chunks in order with the
+// fp32 state held in tensor memory.
 //
 // Method: the chunked parallel mode of "解密Qwen3-Next的Gated DeltaNet：如何用75%混合层实现长文本
 // 高效推理" §2.2 (parallel inside a chunk, the state carried from chunk to chunk) for the gated
