@@ -19,13 +19,18 @@
 namespace gdn {
 namespace {
 
-constexpr int PX_THREADS = 64;  // each thread: 4 rows x 8 columns of the block's 16 x 128 result
+// four groups of 64 threads split the inner dimension (32 of its 128 terms each); a thread of a
+// group: 4 rows x 8 columns of the block's 16 x 128 result
+constexpr int PX_GROUPS = 4;
+constexpr int PX_THREADS = 64 * PX_GROUPS;
 constexpr int PX_ROWS = 16;
-constexpr size_t PX_SMEM = (2 * (size_t)tm::D * tm::D + PX_ROWS * tm::D) * sizeof(float);
+constexpr size_t PX_SMEM =
+    (2 * (size_t)tm::D * tm::D + (size_t)PX_GROUPS * PX_ROWS * tm::D) * sizeof(float);
 
 // M_k comes in by one bulk copy per step into alternating buffers, the next one while the current
 // step computes; the running rows stay in shared memory.  Register blocking (4 rows per thread)
-// keeps the inner product off the shared-memory port.
+// keeps the inner product off the shared-memory port: each M element is read once per group and
+// the groups cover disjoint rows of M, so the block reads M once per step.
 __global__ void __launch_bounds__(PX_THREADS) scan_prefix_kernel(
     const int32_t* __restrict__ cu, int64_t T, int N, int Hv, const int64_t* __restrict__ plan,
     int64_t max_segs, float* __restrict__ st, int* status) {
@@ -33,6 +38,7 @@ __global__ void __launch_bounds__(PX_THREADS) scan_prefix_kernel(
   extern __shared__ __align__(16) float px_smem[];
   float* Ms = px_smem;                     // two buffers of M (128 x 128)
   float* Sr = Ms + 2 * tm::D * tm::D;      // the block's 16 rows of the running state
+  float* Pp = Sr + PX_ROWS * tm::D;         // partial sums of groups 1..3
   __shared__ uint64_t bars[3];             // M buffer 0, M buffer 1, first rows
   const int n = blockIdx.x, h = blockIdx.y, r0 = PX_ROWS * blockIdx.z;
   const int tid = threadIdx.x;
@@ -77,7 +83,9 @@ __global__ void __launch_bounds__(PX_THREADS) scan_prefix_kernel(
   }
   // every request made is waited for before the CTA can leave (bounded waits)
   bool ok = ptx::mbar_wait(&bars[2], 0);
-  const int rg = tid >> 4, c0 = 8 * (tid & 15);  // rows 4 rg .. 4 rg + 3, columns c0 .. c0 + 7
+  const int kg = tid >> 6, tt = tid & 63;          // inner-dimension group, thread in the group
+  const int rg = tt >> 4, c0 = 8 * (tt & 15);      // rows 4 rg .. 4 rg + 3, columns c0 .. c0 + 7
+  constexpr int LK = tm::D / PX_GROUPS;            // inner terms per group
   for (int64_t k = 1; k < nseg; ++k) {
     if (__syncthreads_and(ok)) {
       for (int e = tid; e < PX_ROWS * tm::D / 4; e += PX_THREADS)
@@ -91,18 +99,23 @@ __global__ void __launch_bounds__(PX_THREADS) scan_prefix_kernel(
     float acc[4][8];
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      const float4* b4 =
-          reinterpret_cast<const float4*>(bseg + g_of(k) + (size_t)(r0 + 4 * rg + i) * tm::D + c0);
-      const float4 x0 = b4[0], x1 = b4[1];
-      acc[i][0] = x0.x; acc[i][1] = x0.y; acc[i][2] = x0.z; acc[i][3] = x0.w;
-      acc[i][4] = x1.x; acc[i][5] = x1.y; acc[i][6] = x1.z; acc[i][7] = x1.w;
+      if (kg == 0) {  // group 0 starts from B_k, the others from zero
+        const float4* b4 = reinterpret_cast<const float4*>(bseg + g_of(k) +
+                                                           (size_t)(r0 + 4 * rg + i) * tm::D + c0);
+        const float4 x0 = b4[0], x1 = b4[1];
+        acc[i][0] = x0.x; acc[i][1] = x0.y; acc[i][2] = x0.z; acc[i][3] = x0.w;
+        acc[i][4] = x1.x; acc[i][5] = x1.y; acc[i][6] = x1.z; acc[i][7] = x1.w;
+      } else {
+#pragma unroll
+        for (int q = 0; q < 8; ++q) acc[i][q] = 0.0f;
+      }
     }
     const bool have = ptx::mbar_wait(&bars[buf], (uint32_t)((k - 1) >> 1) & 1);
     ok = ok && have;
     if (__syncthreads_and(ok)) {
       const float* M = Ms + buf * tm::D * tm::D;
 #pragma unroll 4
-      for (int l = 0; l < tm::D; ++l) {
+      for (int l = LK * kg; l < LK * (kg + 1); ++l) {
         const float4 m0 = *reinterpret_cast<const float4*>(M + l * tm::D + c0);
         const float4 m1 = *reinterpret_cast<const float4*>(M + l * tm::D + c0 + 4);
 #pragma unroll
@@ -114,12 +127,24 @@ __global__ void __launch_bounds__(PX_THREADS) scan_prefix_kernel(
           acc[i][6] = fmaf(sv, m1.z, acc[i][6]); acc[i][7] = fmaf(sv, m1.w, acc[i][7]);
         }
       }
+      if (kg > 0) {
+        float* pp = Pp + (size_t)(kg - 1) * PX_ROWS * tm::D;
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+          for (int q = 0; q < 8; ++q) pp[(4 * rg + i) * tm::D + c0 + q] = acc[i][q];
+      }
     }
-    __syncthreads();  // Sr and this M buffer have been read by every thread
+    __syncthreads();  // Sr and this M buffer have been read by every thread; partials written
+    if (kg == 0) {
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
+      for (int i = 0; i < 4; ++i)
 #pragma unroll
-      for (int q = 0; q < 8; ++q) Sr[(4 * rg + i) * tm::D + c0 + q] = acc[i][q];
+        for (int q = 0; q < 8; ++q) {
+          const int e = (4 * rg + i) * tm::D + c0 + q;
+          Sr[e] = acc[i][q] + (Pp[e] + Pp[PX_ROWS * tm::D + e]) + Pp[2 * PX_ROWS * tm::D + e];
+        }
+    }
   }
   if (!ok && tid == 0) report(status, GDN_ERR_TIMEOUT);
 }
