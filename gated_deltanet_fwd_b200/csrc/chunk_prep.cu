@@ -42,7 +42,8 @@ constexpr uint32_t PP_MB = PP_T + PAIR * 64 * AS * 4;         // PAIR x 4 x fp32
 constexpr uint32_t PP_GB = PP_MB + PAIR * 4 * 16 * MS * 4;    // PAIR x (gamma log2e [64], beta [64])
 constexpr uint32_t PP_BAR = PP_GB + PAIR * 128 * 4;           // mbarrier, tensor-memory slot
 constexpr uint32_t PP_SMEM = PP_BAR + 64 + 1024;              // + slack for 1024-byte alignment
-static_assert(PP_SMEM <= 115 * 1024, "two prep CTAs per SM");
+// two CTAs per SM: the SM's 228 KB of shared memory less 1 KB the hardware reserves per CTA
+static_assert(PP_SMEM <= 228 * 1024 / 2 - 1024, "two prep CTAs per SM");
 
 constexpr float kLog2e = 1.4426950408889634f;
 
